@@ -1,0 +1,188 @@
+"""Python binding of libbsa: Top-p block routing + block-sparse attention on B200.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+libbsa.so (csrc/).  PyTorch supplies device memory and streams.  If the
+library is missing the import fails loudly; there is no CPU path.
+
+The functions keep the C names (bsa_route, bsa_sparse_attn, ...) and take
+torch tensors where the C call takes device pointers; `Plan` wraps
+bsa_plan_create / bsa_plan_destroy.  `route` and `sparse_attn` are thin
+conveniences that allocate the outputs and the workspace with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libbsa.so not built at {LIB_PATH}: run `python -m block_sparse_attention_top_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+BSA_OK, BSA_EINVAL, BSA_EUNSUPPORTED, BSA_ECAPACITY, BSA_EWORKSPACE, BSA_ECUDA, BSA_EDEVICE = 0, -1, -2, -3, -4, -5, -6
+BSA_ORDER_HILBERT2D_FRAME, BSA_ORDER_IDENTITY = 0, 1
+BSA_BF16, BSA_F32 = 0, 1
+BSA_OP_ROUTE, BSA_OP_ATTN = 0, 1
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+_SIGS = {
+    "bsa_plan_create": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _I]),
+    "bsa_plan_destroy": (None, [_P]),
+    "bsa_plan_info": (_I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
+    "bsa_token_order": (_I, [_I, _I, _I, _I, _P]),
+    "bsa_workspace_size": (_SZ, [_P, _I]),
+    "bsa_route": (_I, [_P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
+    "bsa_route_intermediates": (_I, [_P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P)]),
+    "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_attn_run": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_attn_run_simt": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_last_device_error": (_I, [_P, _P]),
+    "bsa_strerror": (ctypes.c_char_p, [_I]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {bsa_strerror(status)} ({status})")
+        self.status = status
+
+
+def bsa_strerror(status: int) -> str:
+    return _lib.bsa_strerror(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != BSA_OK:
+        raise BsaError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Plan:
+    """Owns a bsa_plan for one (B, H, T, Hs, Ws, head_dim, block, order) shape."""
+
+    def __init__(self, B, H, T, Hs, Ws, head_dim, block, order=BSA_ORDER_HILBERT2D_FRAME):
+        h = _P()
+        _check(_lib.bsa_plan_create(ctypes.byref(h), B, H, T, Hs, Ws, head_dim, block, order), "bsa_plan_create")
+        self.handle = h
+        self.B, self.H, self.T, self.Hs, self.Ws, self.d, self.block, self.order = B, H, T, Hs, Ws, head_dim, block, order
+        n, nb, rows = _I64(), _I64(), _I64()
+        _check(_lib.bsa_plan_info(h, ctypes.byref(n), ctypes.byref(nb), ctypes.byref(rows)), "bsa_plan_info")
+        self.N, self.nb, self.rows = n.value, nb.value, rows.value
+
+    def workspace_size(self, op: int) -> int:
+        return int(_lib.bsa_workspace_size(self.handle, op))
+
+    def workspace(self, op: int, device="cuda") -> torch.Tensor:
+        return torch.empty(self.workspace_size(op), dtype=torch.uint8, device=device)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _lib.bsa_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def bsa_token_order(T: int, Hs: int, Ws: int, order: int = BSA_ORDER_HILBERT2D_FRAME):
+    """Host-only token permutation (int32 CPU tensor)."""
+    out = torch.empty(T * Hs * Ws, dtype=torch.int32)
+    _check(_lib.bsa_token_order(T, Hs, Ws, order, out.data_ptr()), "bsa_token_order")
+    return out
+
+
+def bsa_route(plan, q, k, dtype, p, k_floor, row_ptr, col_idx, col_cap, L_h, nnz, workspace, stream=None):
+    return _lib.bsa_route(plan.handle, _ptr(q), _ptr(k), dtype, float(p), int(k_floor), _ptr(row_ptr),
+                          _ptr(col_idx), int(col_cap), _ptr(L_h), _ptr(nnz), _ptr(workspace),
+                          workspace.numel() if workspace is not None else 0, _stream(stream))
+
+
+def bsa_route_intermediates(plan, workspace):
+    a, b, c = _P(), _P(), _P()
+    _check(_lib.bsa_route_intermediates(plan.handle, _ptr(workspace), ctypes.byref(a), ctypes.byref(b),
+                                        ctypes.byref(c)), "bsa_route_intermediates")
+    return a.value, b.value, c.value
+
+
+def bsa_sparse_attn(plan, q, k, v, row_ptr, col_idx, o, workspace, stream=None):
+    return _lib.bsa_sparse_attn(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), _ptr(o),
+                                _ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def bsa_attn_prepare(plan, q, k, v, row_ptr, workspace, stream=None):
+    return _lib.bsa_attn_prepare(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+
+
+def bsa_attn_run(plan, row_ptr, col_idx, o, workspace, stream=None):
+    return _lib.bsa_attn_run(plan.handle, _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(workspace),
+                             workspace.numel(), _stream(stream))
+
+
+def bsa_attn_run_simt(plan, row_ptr, col_idx, o, workspace, stream=None):
+    return _lib.bsa_attn_run_simt(plan.handle, _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+
+
+def bsa_last_device_error(plan, stream=None) -> int:
+    return _lib.bsa_last_device_error(plan.handle, _stream(stream))
+
+
+# ---- conveniences (allocate outputs with torch, raise on error) ----
+
+def route(plan: Plan, q: torch.Tensor, k: torch.Tensor, p: float, k_floor: int, workspace=None,
+          col_cap: int | None = None, stream=None):
+    """Returns (row_ptr, col_idx[:col_cap], L_h, nnz) device tensors; nnz stays on device."""
+    dev = q.device
+    dtype = BSA_BF16 if q.dtype == torch.bfloat16 else BSA_F32
+    if col_cap is None:
+        col_cap = plan.rows * plan.nb
+    row_ptr = torch.empty(plan.rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(col_cap, 1), dtype=torch.int32, device=dev)
+    L_h = torch.empty(plan.B * plan.H, dtype=torch.float32, device=dev)
+    nnz = torch.empty(1, dtype=torch.int64, device=dev)
+    if workspace is None:
+        workspace = plan.workspace(BSA_OP_ROUTE, dev)
+    _check(bsa_route(plan, q, k, dtype, p, k_floor, row_ptr, col_idx, col_cap, L_h, nnz, workspace, stream),
+           "bsa_route")
+    return row_ptr, col_idx, L_h, nnz
+
+
+def sparse_attn(plan: Plan, q, k, v, row_ptr, col_idx, workspace=None, out=None, stream=None):
+    """O = block-sparse attention of bf16 [B,N,H,d] inputs under the CSR mask."""
+    if workspace is None:
+        workspace = plan.workspace(BSA_OP_ATTN, q.device)
+    o = torch.empty_like(q) if out is None else out
+    _check(bsa_sparse_attn(plan, q, k, v, row_ptr, col_idx, o, workspace, stream), "bsa_sparse_attn")
+    return o

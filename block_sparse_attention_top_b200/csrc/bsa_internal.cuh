@@ -1,0 +1,68 @@
+// Internal declarations shared by the libbsa translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/bsa.h"
+
+struct bsa_plan {
+    int B, H, T, Hs, Ws, d, block, order;
+    int64_t N, nb, rows;
+    int device;
+    int num_sms;
+    int32_t* d_perm;     // [N] raster index at reordered position
+    int32_t* d_err;      // [4]: status, detail, spare, spare
+};
+
+namespace bsa {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxRouteBlocks = 8192;   // nb limit of the routing sort
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ---- route workspace layout (offsets in bytes) ----
+struct RouteWs {
+    size_t qbar, kbar, scores, sorted, counts, total;
+};
+RouteWs route_ws_layout(const bsa_plan& p);
+
+// ---- attention workspace layout ----
+struct AttnWs {
+    size_t qp, kp, vp, work, hist, bins, counter, total;
+};
+AttnWs attn_ws_layout(const bsa_plan& p);
+
+// Device error recording: first status wins; detail holds an index.
+__device__ __forceinline__ void record_error(int32_t* err, int status, int detail) {
+    if (atomicCAS(err, 0, status) == 0) err[1] = detail;
+}
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_pool(const bsa_plan& p, const void* q, const void* k, int dtype,
+                        double* qbar, double* kbar, cudaStream_t s);
+cudaError_t launch_scores(const bsa_plan& p, const double* qbar, const double* kbar,
+                          double* scores, cudaStream_t s);
+cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pval, int k_floor,
+                              uint16_t* sorted, int32_t* counts, cudaStream_t s);
+cudaError_t launch_csr(const bsa_plan& p, const int32_t* counts, const uint16_t* sorted,
+                       int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, float* L_h,
+                       int64_t* nnz, cudaStream_t s);
+
+cudaError_t launch_worklist(const bsa_plan& p, const int32_t* row_ptr, int32_t* hist,
+                            int32_t* bins, int32_t* work, cudaStream_t s);
+cudaError_t launch_permute(const bsa_plan& p, const void* q, const void* k, const void* v,
+                           void* qp, void* kp, void* vp, cudaStream_t s);
+cudaError_t launch_attn_simt(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
+                             const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work,
+                             void* o, cudaStream_t s);
+cudaError_t launch_attn_tc(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
+                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work,
+                           int32_t* counter, void* o, cudaStream_t s);
+
+// Host-side token order (no CUDA).
+void token_order(int T, int Hs, int Ws, int order, int32_t* perm);
+
+}  // namespace bsa

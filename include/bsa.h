@@ -1,0 +1,187 @@
+/*
+ * bsa.h -- C ABI of libbsa: Top-p block routing and block-sparse attention
+ * for video diffusion transformers, hand-written for B200 (sm_100a).
+ *
+ * What it computes follows the FVAttn pages:
+ *   - routing: FVAttn review, section 3 "Stage 1: Sparse Mask Routing" and
+ *     section 3.1 "Sparse Routing Frontend" (Hilbert block reordering, Top-p
+ *     CDF threshold, Top-k safety floor, per-head workload and key-block
+ *     importance order); alanhou.org blog, "Key Concepts" (the minimum number
+ *     of blocks whose cumulative attention weight reaches p, and at least k
+ *     blocks); the workload L_h is the review's Eq. 1;
+ *   - attention: FVAttn review, section 3 "Block-Sparse Attention Execution"
+ *     (attention over the retained blocks, then head-order / token-order
+ *     restoration).
+ *
+ * Conventions shared by every call
+ *   - Q, K, V, O: [B, N, H, d] row-major (d fastest), N = T*Hs*Ws tokens in
+ *     raster order (frame, row, column).  d (head_dim) is 64 or 128.
+ *   - Blocks: the tokens are reordered (frame-major 2-D Hilbert order, or
+ *     identity) and cut into nb = ceil(N / block) blocks of `block` tokens;
+ *     the last block holds N - (nb-1)*block tokens.  block is 64 or 128.
+ *   - Mask rows: r = (b*H + h)*nb + i, i a query block; columns j are key
+ *     blocks of the same order.  A mask is CSR: row_ptr int32 [rows+1]
+ *     (row_ptr[0] = 0, non-decreasing), col_idx int32 [nnz], columns unique
+ *     and in [0, nb).  Routed masks list each row's columns in importance
+ *     order (descending block mass); user masks may use any order.
+ *   - Pointers named q, k, v, o, row_ptr, col_idx, L_h, nnz, workspace are
+ *     DEVICE pointers on the plan's device, 16-byte aligned (workspace:
+ *     256-byte aligned).  The caller owns all of them.  `stream` is a
+ *     cudaStream_t (NULL = legacy default stream).
+ *   - Every call returns BSA_OK or a negative status.  Argument errors are
+ *     reported before anything is launched.  Launches are asynchronous on
+ *     `stream`: faults found by the kernels themselves (a malformed mask, a
+ *     too-small col_cap, an expired bounded wait) are recorded in the plan's
+ *     device error word and read with bsa_last_device_error; no kernel traps.
+ *   - A plan may be used from one stream at a time (its device error word
+ *     and the workspace are per call).
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define BSA_OK            0
+#define BSA_EINVAL       -1   /* bad argument (null/unaligned pointer, p outside (0,1], ...) */
+#define BSA_EUNSUPPORTED -2   /* valid but unsupported shape, or not an sm_100 device */
+#define BSA_ECAPACITY    -3   /* routed nnz exceeded col_cap (device-detected) */
+#define BSA_EWORKSPACE   -4   /* workspace missing, too small or misaligned */
+#define BSA_ECUDA        -5   /* a CUDA runtime call or launch failed */
+#define BSA_EDEVICE      -6   /* a kernel found malformed input or a bounded wait expired */
+
+/* ---- token orders ---- */
+#define BSA_ORDER_HILBERT2D_FRAME 0   /* frames in time order; 2-D Hilbert curve inside each frame */
+#define BSA_ORDER_IDENTITY        1   /* raster order */
+
+/* ---- input dtypes for routing ---- */
+#define BSA_BF16 0
+#define BSA_F32  1
+
+/* ---- workspace queries ---- */
+#define BSA_OP_ROUTE 0
+#define BSA_OP_ATTN  1
+
+typedef struct bsa_plan bsa_plan;
+
+/*
+ * Create a plan for one attention shape on the current CUDA device.
+ * Builds the token permutation (perm[n'] = raster index at reordered
+ * position n') on the host and keeps it, and a device error word, on the
+ * device.  Order BSA_ORDER_HILBERT2D_FRAME follows the FVAttn review, section
+ * 3.1 (Hilbert curve block reordering); inside a frame the cells follow the
+ * classic 2-D Hilbert curve over the smallest 2^m square covering Hs x Ws
+ * (x = column, y = row, starting at (0,0), ending at (2^m-1, 0)), skipping
+ * cells outside the grid.
+ * Returns BSA_EINVAL / BSA_EUNSUPPORTED for bad shapes (checked before any
+ * CUDA call), BSA_ECUDA if the device allocation fails.  *out is NULL on error.
+ * Ownership: the plan owns its host struct and device tables; free with
+ * bsa_plan_destroy.
+ */
+int bsa_plan_create(bsa_plan** out, int B, int H, int T, int Hs, int Ws,
+                    int head_dim, int block, int order);
+void bsa_plan_destroy(bsa_plan* plan);
+
+/* Host-only shape query: N tokens, nb blocks per head, rows = B*H*nb. */
+int bsa_plan_info(const bsa_plan* plan, int64_t* N, int64_t* nb, int64_t* rows);
+
+/*
+ * Host-only: write the token permutation of a (T, Hs, Ws) grid under `order`
+ * into perm[0 .. T*Hs*Ws) (caller-owned host memory).  No CUDA call.
+ */
+int bsa_token_order(int T, int Hs, int Ws, int order, int32_t* perm);
+
+/* Bytes of device workspace that bsa_route (BSA_OP_ROUTE) or bsa_sparse_attn
+ * (BSA_OP_ATTN) needs for this plan; 0 for a NULL plan or unknown op. */
+size_t bsa_workspace_size(const bsa_plan* plan, int op);
+
+/*
+ * Top-p block routing (the pages' Stage 1).  Per row r = (b,h,i):
+ *   Qbar_i, Kbar_j = means of Q, K over the real tokens of block i, j
+ *                    (fp64 sums of the input values);
+ *   s_ij = <Qbar_i, Kbar_j> / sqrt(d);  P_ij = softmax_j s_ij   (fp64);
+ *   order j by P descending (equal P: ascending j);
+ *   n_p  = smallest n whose cumulative mass reaches p (n_p = nb if p >= 1 or
+ *          if no prefix reaches p);
+ *   n_i  = min(nb, max(k_floor, n_p)) (the Top-k safety floor);
+ *   row r of the CSR = the first n_i blocks of that order.
+ * Outputs (device): row_ptr int32 [rows+1]; col_idx int32 [col_cap];
+ * L_h float [B*H] = (sum_i n_i) / nb (the review's Eq. 1); nnz int64 [1].
+ * q, k: [B,N,H,d] of `dtype` (BSA_BF16 or BSA_F32).  p in (0, 1];
+ * k_floor >= 0.  col_cap = B*H*nb*nb can never overflow; if the routed nnz
+ * exceeds col_cap the columns past col_cap are dropped and the device error
+ * word becomes BSA_ECAPACITY.  Needs nb <= 8192 (BSA_EUNSUPPORTED otherwise).
+ * workspace: >= bsa_workspace_size(plan, BSA_OP_ROUTE) bytes, 256-aligned.
+ */
+int bsa_route(const bsa_plan* plan, const void* q, const void* k, int dtype,
+              float p, int k_floor,
+              int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
+              float* L_h, int64_t* nnz,
+              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Device pointers to the intermediates the last bsa_route left in
+ * `workspace`: pooled Qbar and Kbar, fp64 [B*H, nb, d]; block scores
+ * s_ij, fp64 [B*H, nb, nb].  For tests and diagnostics; no CUDA call.
+ */
+int bsa_route_intermediates(const bsa_plan* plan, void* workspace,
+                            const double** qbar, const double** kbar,
+                            const double** scores);
+
+/*
+ * Block-sparse attention (the pages' "Block-Sparse Attention Execution"):
+ *   O[b, n, h, :] = sum over the real tokens t of the key blocks listed in
+ *   row (b,h,i) of softmax_t(Q[b,n,h,:] . K[b,t,h,:] / sqrt(d)) V[b,t,h,:]
+ * for every token n of query block i, non-causal, written back in raster
+ * token order.  Rows with no key block produce zeros.
+ * q, k, v, o: bf16 [B,N,H,d]; row_ptr/col_idx: a CSR mask as above.
+ * Equivalent to bsa_attn_prepare followed by bsa_attn_run on `stream`.
+ * A column outside [0, nb) or a decreasing row_ptr is skipped and recorded
+ * as BSA_EDEVICE in the device error word.
+ * workspace: >= bsa_workspace_size(plan, BSA_OP_ATTN) bytes, 256-aligned.
+ */
+int bsa_sparse_attn(const bsa_plan* plan, const void* q, const void* k, const void* v,
+                    const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The two halves of bsa_sparse_attn, for callers that time or overlap them.
+ * prepare: orders the work items (b,h,i) heaviest first by their number of
+ *   key blocks, and copies Q, K, V into reordered, zero-padded
+ *   [B, H, nb*block, d] bf16 tiles inside the workspace.
+ * run: the persistent tcgen05 attention kernel over that work list; writes O.
+ * run must follow prepare on the same stream with the same workspace.
+ */
+int bsa_attn_prepare(const bsa_plan* plan, const void* q, const void* k, const void* v,
+                     const int32_t* row_ptr, void* workspace, size_t ws_bytes, void* stream);
+int bsa_attn_run(const bsa_plan* plan, const int32_t* row_ptr, const int32_t* col_idx,
+                 void* o, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Same contract as bsa_attn_run, computed by a slow CUDA-core kernel (one
+ * warp per query token, fp32 online softmax).  A cross-check for the
+ * tensor-core kernel in tests; not a performance path.
+ */
+int bsa_attn_run_simt(const bsa_plan* plan, const int32_t* row_ptr, const int32_t* col_idx,
+                      void* o, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the plan's device error word.
+ * Returns BSA_OK, or the first device-side status recorded since the last
+ * call (BSA_ECAPACITY, BSA_EDEVICE), or BSA_ECUDA if the stream itself
+ * reports an error.
+ */
+int bsa_last_device_error(const bsa_plan* plan, void* stream);
+
+/* Static description of a status code. */
+const char* bsa_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H */

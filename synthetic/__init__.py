@@ -188,3 +188,9 @@ def window_anchor_mask(w: Workload, step: int = 0, radius: int = 2, n_anchor: in
     row_ptr = np.zeros(reps * nb + 1, dtype=np.int64)
     row_ptr[1:] = np.cumsum(np.tile(counts, reps))
     return row_ptr.astype(np.int32), np.tile(cols, reps)
+
+
+def seed_for(cid: int, p_index: int = 0) -> int:
+    """Seed of config `cid` at its `p_index`-th Top-p value: 1000*cid + 1 + p_index
+    (config 3: 3001/3002/3003 for p = 0.8/0.9/0.95)."""
+    return 1000 * cid + 1 + p_index

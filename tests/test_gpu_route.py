@@ -1,0 +1,138 @@
+"""GPU routing (bsa_route) against the oracle: masks bit-exact outside the
+tie set, intermediates, edge cases and error paths."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as syn
+from _gpu import to_dev
+from _parity import check_route
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    from block_sparse_attention_top_b200 import build
+    build.build()
+    import block_sparse_attention_top_b200 as m
+    return m
+
+
+def gpu_route(bsa, w, x, p, k_floor, order=0, col_cap=None):
+    plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block, order)
+    q, k = to_dev(x["q"]), to_dev(x["k"])
+    ws = plan.workspace(bsa.BSA_OP_ROUTE)
+    rp, ci, L, nnz = bsa.route(plan, q, k, p, k_floor, workspace=ws, col_cap=col_cap)
+    status = bsa.bsa_last_device_error(plan)
+    out = dict(row_ptr=rp.cpu().numpy(), col_idx=ci.cpu().numpy(), L_h=L.cpu().numpy(),
+               nnz=int(nnz.item()), status=status, plan=plan, ws=ws)
+    return out
+
+
+def compare(bsa, w, x, p, k_floor, order=0):
+    ref = oracle.route(x["q"], x["k"], w.T, w.Hs, w.Ws, w.block, p, k_floor,
+                       order="hilbert" if order == 0 else "identity")
+    g = gpu_route(bsa, w, x, p, k_floor, order)
+    assert g["status"] == 0
+    amb = check_route(g["row_ptr"], g["col_idx"], g["L_h"], g["nnz"], ref, w.B * w.H)
+    assert amb < 0.01 or w.rows < 1000        # tie fraction only meaningful on many rows
+    return g, ref
+
+
+def _fetch(ws, ptr, n):
+    """fp64 [n] view of the workspace at device address `ptr`, copied to host."""
+    off = ptr - ws.data_ptr()
+    assert 0 <= off and off + 8 * n <= ws.numel()
+    return ws[off:off + 8 * n].view(torch.float64).cpu().numpy()
+
+
+@pytest.mark.parametrize("p,k_floor", [(0.9, 2), (0.5, 0), (1.0, 0), (0.9, 16), (0.3, 40), (1e-4, 3)])
+def test_tiny_full(bsa, p, k_floor):
+    w = syn.workload(1)
+    compare(bsa, w, syn.make_inputs(w, seed=syn.seed_for(1)), p, k_floor)
+
+
+def test_intermediates_exact(bsa):
+    """Pooled means are exact fp64 sums / m on both sides (bf16 inputs sum exactly)."""
+    w = syn.workload(2, T=3, Hs=30, Ws=52)
+    x = syn.make_inputs(w, seed=77)
+    g, ref = compare(bsa, w, x, 0.9, 4)
+    qb, kb, sc = bsa.bsa_route_intermediates(g["plan"], g["ws"])
+    n = w.B * w.H * w.nb
+    qbar = _fetch(g["ws"], qb, n * w.d).reshape(ref.qbar.shape)
+    kbar = _fetch(g["ws"], kb, n * w.d).reshape(ref.kbar.shape)
+    scores = _fetch(g["ws"], sc, n * w.nb).reshape(ref.scores.shape)
+    assert np.array_equal(qbar, ref.qbar) and np.array_equal(kbar, ref.kbar)
+    assert np.abs(scores - ref.scores).max() <= 1e-12 * max(1.0, np.abs(ref.scores).max())
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=1, Hs=5, Ws=7, H=3, d=64, block=64),      # N=35 < block: one ragged block
+    dict(T=3, Hs=7, Ws=9, H=2, d=128, block=64),     # N=189: tail of 61
+    dict(T=2, Hs=33, Ws=17, H=1, d=64, block=128),   # non-square, tail of augmented
+    dict(T=5, Hs=16, Ws=16, H=4, d=128, block=128),  # exact multiple
+])
+@pytest.mark.parametrize("order", [0, 1])
+def test_ragged_shapes(bsa, shape, order):
+    w = syn.workload(2, **shape)
+    x = syn.make_inputs(w, seed=11)
+    for p, kf in ((0.9, 2), (0.7, 0), (1.0, 1)):
+        compare(bsa, w, x, p, kf, order)
+
+
+def test_fp32_input_path(bsa):
+    w = syn.workload(1, T=2, Hs=12, Ws=20, H=3)
+    x = syn.make_inputs(w, seed=5)
+    assert x["q"].dtype == np.float32
+    compare(bsa, w, x, 0.8, 2)
+
+
+@pytest.mark.parametrize("cid,p_index", [(2, 0), (3, 0), (3, 1), (3, 2), (4, 0)])
+def test_full_size_configs(bsa, cid, p_index):
+    w = syn.workload(cid)
+    x = syn.make_inputs(w, seed=syn.seed_for(cid, p_index))
+    g, ref = compare(bsa, w, x, w.ps[p_index], w.k_floor)
+    print(f"config {cid} p={w.ps[p_index]}: density {ref.nnz / (w.rows * w.nb):.3f}, "
+          f"ambiguous rows {int(ref.ambiguous.sum())}/{w.rows}")
+
+
+def test_capacity_overflow_is_reported(bsa):
+    w = syn.workload(1)
+    x = syn.make_inputs(w, seed=3)
+    g = gpu_route(bsa, w, x, 0.9, 2, col_cap=10)
+    assert g["status"] == bsa.BSA_ECAPACITY
+    assert g["nnz"] > 10
+    assert bsa.bsa_last_device_error(g["plan"]) == 0          # cleared after reading
+
+
+def test_argument_errors(bsa):
+    w = syn.workload(1)
+    plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block)
+    x = syn.make_inputs(w, seed=3)
+    q, k = to_dev(x["q"]), to_dev(x["k"])
+    rp = torch.empty(plan.rows + 1, dtype=torch.int32, device="cuda")
+    ci = torch.empty(plan.rows * plan.nb, dtype=torch.int32, device="cuda")
+    L = torch.empty(plan.B * plan.H, device="cuda")
+    nnz = torch.empty(1, dtype=torch.int64, device="cuda")
+    ws = plan.workspace(bsa.BSA_OP_ROUTE)
+    call = lambda **kw: bsa.bsa_route(plan, kw.get("q", q), k, bsa.BSA_F32, kw.get("p", 0.9), kw.get("kf", 1), rp, ci,
+                                      ci.numel(), L, nnz, kw.get("ws", ws))
+    assert call() == 0
+    assert call(p=0.0) == bsa.BSA_EINVAL
+    assert call(p=1.5) == bsa.BSA_EINVAL
+    assert call(p=float("nan")) == bsa.BSA_EINVAL
+    assert call(kf=-1) == bsa.BSA_EINVAL
+    assert call(q=q.data_ptr() + 4) == bsa.BSA_EINVAL
+    assert call(ws=ws[: ws.numel() - 1024]) == bsa.BSA_EWORKSPACE
+    assert bsa.bsa_last_device_error(plan) == 0
+
+
+def test_too_many_blocks_unsupported(bsa):
+    plan = bsa.Plan(1, 1, 1, 1025, 1025, 64, 64)      # nb = 16417 > 8192
+    assert plan.nb > 8192
+    d = torch.empty(16, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    assert bsa.bsa_route(plan, d, d, bsa.BSA_F32, 0.9, 1, d, d, 0, d, torch.empty(1, dtype=torch.int64, device="cuda"),
+                         ws) == bsa.BSA_EUNSUPPORTED
