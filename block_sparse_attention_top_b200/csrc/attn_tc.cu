@@ -4,21 +4,27 @@
 //
 // One CTA per SM walks a static zig-zag share of the heaviest-first work list
 // (one item = one 128-row query tile of one head).  Per item and retained key
-// block j, with S and O living in tensor memory (TMEM):
+// block j, with S, P and O living in tensor memory (TMEM):
 //
 //   warp 0 (1 thread)   TMA: Q tile once per item; K_j, V_j into 2-stage rings
-//   warp 1 (1 thread)   tcgen05.mma: S[j%2] = Q K_j^T   (M=128, N=block, K=d)
-//                                    O     += P_j V_j   (M=128, N=d,     K=block)
-//   warps 2..5          softmax: thread = query row = TMEM lane; reads S[j%2]
-//                       (tcgen05.ld), online softmax in the log2 domain, writes
-//                       P_j (bf16) into a 128B-swizzled shared tile, rescales the
-//                       O row in TMEM only when its running max grows by more
-//                       than 2^8; epilogue: O / l, bf16, stored at the token's
-//                       raster position (the inverse Hilbert permutation is
-//                       fused into this store).
+//   warp 1 (1 thread)   tcgen05.mma: S[j%2] = Q K_j^T      (M=128, N=block, K=d; A, B in smem)
+//                                    O     += P[j%2] V_j   (M=128, N=d, K=block; P in TMEM)
+//   warps 2..9          softmax: TMEM lane = query row; each row is split over
+//                       two warps, one per half of the key (and output)
+//                       columns.  Both read the whole S row for its maximum, so
+//                       no exchange is needed per block.  Online softmax in the
+//                       log2 domain; a quarter of the exponentials run as a
+//                       polynomial on the FMA pipe to offload the MUFU unit;
+//                       P_j goes to its own TMEM columns as bf16 pairs
+//                       (tcgen05.st); the O row is rescaled in TMEM only when
+//                       its running max grows by more than 2^8.  Epilogue: the
+//                       two partial row sums meet through shared memory, then
+//                       O / l, bf16, stored at the token's raster position (the
+//                       inverse Hilbert permutation is fused into this store).
 //
-// S is double-buffered, so QK^T of block j+1 and PV of block j-1 run on the
-// tensor pipe while the softmax warps work on block j.
+// S and P are double-buffered, so QK^T of block j+1 and PV of block j-1 run
+// on the tensor pipe while the softmax warps work on block j.  TMEM columns:
+// S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
 //
 // Every wait on an mbarrier is bounded (about 4 s of %globaltimer); on expiry
 // the CTA records BSA_EDEVICE, raises a shared abort flag that stops the other
@@ -34,10 +40,11 @@
 namespace bsa {
 namespace {
 
-constexpr int kThreads = 192;           // 6 warps
-constexpr int kTileM = 128;             // query rows per tile (TMEM lanes)
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 32 * (2 + kSoftmaxWarps);   // producer, MMA, softmax
+constexpr int kTileM = 128;                          // query rows per tile (TMEM lanes)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
 // ---------------------------------------------------------------- PTX helpers
@@ -105,8 +112,8 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                  : "memory");
 }
 // D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
@@ -114,28 +121,46 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#define BSA_R8(b) "=r"(r[b + 0]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), \
+                  "=r"(r[b + 4]), "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7])
+#define BSA_W8(b) "r"(r[b + 0]), "r"(r[b + 1]), "r"(r[b + 2]), "r"(r[b + 3]), \
+                  "r"(r[b + 4]), "r"(r[b + 5]), "r"(r[b + 6]), "r"(r[b + 7])
+// 32 lanes x 32 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : BSA_R8(0), BSA_R8(8), BSA_R8(16), BSA_R8(24)
         : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
         "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        ::"r"(taddr), BSA_W8(0), BSA_W8(8), BSA_W8(16), BSA_W8(24)
         : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), BSA_W8(0), BSA_W8(8)
+        : "memory");
+}
+#undef BSA_R8
+#undef BSA_W8
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -145,36 +170,64 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128.
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128,
+// A K-major; B K-major (0) or MN-major (1).
 __host__ __device__ constexpr uint32_t instr_desc(int n, int b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(kTileM >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float ex2_mufu(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+// 2^x on the FMA pipe for x in [-127, 128): split x = j + f with j = rint(x),
+// f in [-1/2, 1/2] (adding 1.5 * 2^23 rounds to an integer held in the low
+// mantissa bits), a degree-3 polynomial for 2^f (coefficients from a
+// relative-error minimax fit on [-1/2, 1/2], max relative error 7.5e-5), and
+// j added straight into the exponent field.  Accurate far beyond the bf16
+// rounding P receives.
+__device__ __forceinline__ float ex2_poly(float x) {
+    x = fmaxf(x, -127.f);
+    const float t = x + 12582912.f;
+    const float j = t - 12582912.f;
+    const float f = x - j;
+    float p = fmaf(0.0551716648f, f, 0.2426111251f);
+    p = fmaf(p, f, 0.6932609677f);
+    p = fmaf(p, f, 0.9999280572f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // ------------------------------------------------------------- shared layout
 template <int D, int BLK>
 struct Smem {
-    static constexpr int kQ = kTileM * D * 2;       // Q tile, D/64 column slabs of 128 rows
-    static constexpr int kKV = BLK * D * 2;         // one K or V tile
-    static constexpr int kP = kTileM * BLK * 2;     // P tile, BLK/64 slabs of 128 rows
+    static constexpr int kQ = kTileM * D * 2;       // Q tile: D/64 slabs of [128 rows x 128 B]
+    static constexpr int kKV = BLK * D * 2;         // one K or V tile: D/64 slabs of [BLK rows x 128 B]
     static constexpr int offQ = 0;
     static constexpr int offK = offQ + kQ;
     static constexpr int offV = offK + 2 * kKV;
-    static constexpr int offP = offV + 2 * kKV;
-    static constexpr int offBar = offP + kP;
-    static constexpr int kBars = 17;
+    static constexpr int offXchg = offV + 2 * kKV;  // float [2 item parity][2 half][128 rows] row sums
+    static constexpr int offBar = offXchg + 2 * 2 * kTileM * 4;
+    static constexpr int kBars = 20;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kBytes = offMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;   // room to align the base to 1024 B
 };
 // barrier slots
 enum { B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0,
-       B_VEMPTY1, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PVDONE, B_DRAIN, B_COUNT };
+       B_VEMPTY1, B_SFULL0, B_SFULL1, B_PFULL, B_PVDONE, B_DRAIN, B_PAIR0, B_PAIR1, B_PAIR2, B_PAIR3,
+       B_COUNT };
 
 struct Params {
     const int32_t* row_ptr;
@@ -200,6 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const Params prm) {
     using L = Smem<D, BLK>;
+    constexpr int HC = BLK / 2;     // S columns per softmax warp
+    constexpr int OC = D / 2;       // O columns per softmax warp
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -208,13 +263,14 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offMisc + 8);
+    float* xchg = reinterpret_cast<float*>(smem + L::offXchg);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(bar(i), (i == B_SEMPTY0 || i == B_SEMPTY1 || i == B_PFULL) ? 128u : 1u);
+            mbar_init(bar(i), i == B_PFULL ? 32u * kSoftmaxWarps : (i >= B_PAIR0 ? 64u : 1u));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (BLK < kTileM) {
@@ -286,17 +342,17 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             constexpr uint32_t idesc_pv = instr_desc(D, 1);
             uint32_t kv_it = 0, q_it = 0, pv_it = 0;
             bool ok = true;
-            // PV of iteration `it` (stage it&1) for the item's local block `first`
+            // O += P V for kv iteration `it`; P sits in TMEM buffer it&1
             auto issue_pv = [&](uint32_t it, bool first) -> bool {
                 if (!mbar_wait(bar(B_PFULL), pv_it & 1, abort_flag)) return false;
                 const int st = it & 1;
                 if (!mbar_wait(bar(B_VFULL0 + st), (it >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint32_t p_tmem = tmem + ((it & 1) ? kColP1 : kColP0);
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t a = smem_desc(sbase + L::offP + (kk / 4) * kTileM * 128 + (kk % 4) * 32, 16, 1024);
                     const uint64_t b = smem_desc(sbase + L::offV + st * L::kKV + kk * 16 * 128, BLK * 128, 1024);
-                    tc_mma(tmem + kColO, a, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                    tc_mma_ts(tmem + kColO, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
                 }
                 tc_commit(bar(B_PVDONE));
                 tc_commit(bar(B_VEMPTY0 + st));
@@ -317,18 +373,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 for (int jj = beg; jj < end && ok; ++jj) {
                     if (!valid_col(prm.col_idx[jj], nb)) continue;
                     const int st = kv_it & 1;
-                    const int sb = kv_it & 1;     // S buffer follows the kv iteration
+                    // S buffer kv_it&1 is free: the softmax warps read S(kv_it-2) before the
+                    // P_FULL arrival that this thread waited on for PV(kv_it-2).
                     if (!(ok = mbar_wait(bar(B_KFULL0 + st), (kv_it >> 1) & 1, abort_flag))) break;
-                    if (kv_it >= 2 && !(ok = mbar_wait(bar(B_SEMPTY0 + sb), ((kv_it >> 1) & 1) ^ 1, abort_flag))) break;
                     tc_fence_after();
-                    const uint32_t d_s = tmem + (sb ? kColS1 : kColS0);
+                    const uint32_t d_s = tmem + ((kv_it & 1) ? kColS1 : kColS0);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t a = smem_desc(sbase + L::offQ + (kk / 4) * kTileM * 128 + (kk % 4) * 32, 16, 1024);
                         const uint64_t b = smem_desc(sbase + L::offK + st * L::kKV + (kk / 4) * BLK * 128 + (kk % 4) * 32, 16, 1024);
-                        tc_mma(d_s, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                        tc_mma_ss(d_s, a, b, idesc_qk, kk > 0 ? 1u : 0u);
                     }
-                    tc_commit(bar(B_SFULL0 + sb));
+                    tc_commit(bar(B_SFULL0 + (kv_it & 1)));
                     tc_commit(bar(B_KEMPTY0 + st));
                     if (local == nvalid - 1) tc_commit(bar(B_QEMPTY));
                     if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
@@ -348,9 +404,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
     } else {
         // ------------------------------------------------------------- softmax
-        const int row = 32 * (warp & 3) + lane;          // TMEM lane == query row in tile
-        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        uint32_t kv_it = 0, pv_it = 0;
+        const int quad = warp & 3;                       // TMEM lane quadrant
+        const int half = (warp - 2) >> 2;                // which half of the key / output columns
+        const int row = 32 * quad + lane;                // TMEM lane == query row in tile
+        const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+        uint32_t kv_it = 0, pv_it = 0, items = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int idx = item_index(k, cta, grid);
@@ -363,11 +421,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const int b = bh / prm.H, h = bh % prm.H;
             const int n_tok = i * BLK + row;             // reordered position of this row
             const bool row_real = row < BLK && n_tok < prm.N;
+            __nv_bfloat16* dst = prm.o + (((int64_t)b * prm.N + (row_real ? prm.perm[n_tok] : 0)) * prm.H + h) * D +
+                                 half * OC;
             if (nvalid == 0) {
-                if (row_real) {
-                    uint4* dst = reinterpret_cast<uint4*>(prm.o + (((int64_t)b * prm.N + prm.perm[n_tok]) * prm.H + h) * D);
-                    for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-                }
+                if (row_real)
+                    for (int c = 0; c < OC / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
                 continue;
             }
             float m_use = 0.f, l = 0.f;
@@ -376,93 +434,128 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const int j = prm.col_idx[jj];
                 if (!valid_col(j, nb)) continue;
                 const int sb = kv_it & 1;
+                const uint32_t s_col = sb ? kColS1 : kColS0;
                 if (!(ok = warp_wait(bar(B_SFULL0 + sb), (kv_it >> 1) & 1, abort_flag))) break;
                 tc_fence_after();
-                float s[BLK];
+                // padding keys of a ragged last block
+                const int valid_keys = prm.N - j * BLK;
+                const bool ragged = valid_keys < BLK;
+                float s[HC];
+                float lm0, lm1;
                 {
-                    uint32_t raw[32];
+                    // the other half: only its maximum is needed
+                    uint32_t raw[HC];
 #pragma unroll
-                    for (int c = 0; c < BLK / 32; ++c) {
-                        tmem_ld32(tmem + lane_base + (sb ? kColS1 : kColS0) + c * 32, raw);
-                        tmem_wait_ld();
+                    for (int c = 0; c < HC / 32; ++c)
+                        tmem_ld32(tmem + lane_base + s_col + (1 - half) * HC + c * 32, raw + 32 * c);
+                    tmem_wait_ld();
+                    if (ragged) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
+                        for (int c = 0; c < HC; ++c)
+                            if ((1 - half) * HC + c >= valid_keys) raw[c] = __float_as_uint(-INFINITY);
                     }
-                }
-                tc_fence_before();
-                mbar_arrive(bar(B_SEMPTY0 + sb));
-                // mask the padding keys of a ragged last block
-                const int valid_keys = min(BLK, prm.N - j * BLK);
-                float mx = -INFINITY;
+                    lm0 = __uint_as_float(raw[0]);
+                    lm1 = __uint_as_float(raw[1]);
 #pragma unroll
-                for (int c = 0; c < BLK; ++c) {
-                    s[c] = c < valid_keys ? s[c] * prm.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
+                    for (int c = 2; c + 1 < HC; c += 4) {
+                        lm0 = max3(lm0, __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
+                        if (c + 3 < HC) lm1 = max3(lm1, __uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3]));
+                    }
+#pragma unroll
+                    for (int c = 0; c < HC / 32; ++c)
+                        tmem_ld32(tmem + lane_base + s_col + half * HC + c * 32, raw + 32 * c);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < HC; ++c) s[c] = __uint_as_float(raw[c]);
                 }
+                if (ragged) {
+#pragma unroll
+                    for (int c = 0; c < HC; ++c)
+                        if (half * HC + c >= valid_keys) s[c] = -INFINITY;
+                }
+#pragma unroll
+                for (int c = 0; c + 1 < HC; c += 4) {
+                    lm0 = max3(lm0, s[c], s[c + 1]);
+                    if (c + 3 < HC) lm1 = max3(lm1, s[c + 2], s[c + 3]);
+                }
+                const float mx = fmaxf(lm0, lm1) * prm.scale_log2;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (local == 0) {
                     m_use = mx;
                 } else if (mx > m_use + 8.f) {
-                    alpha = exp2f(m_use - mx);
+                    alpha = ex2_mufu(m_use - mx);
                     m_use = mx;
                     rescale = true;
                 }
-                float rowsum = 0.f;
-                uint32_t packed[BLK / 2];
+                const float neg_m = -m_use;
+                float sum0 = 0.f, sum1 = 0.f;
+                uint32_t pk[HC / 2];
 #pragma unroll
-                for (int c = 0; c < BLK; c += 2) {
-                    const float p0 = exp2f(s[c] - m_use);
-                    const float p1 = exp2f(s[c + 1] - m_use);
-                    rowsum += p0 + p1;
-                    packed[c / 2] = pack_bf16(p0, p1);
+                for (int c = 0; c < HC; c += 2) {
+                    const float x0 = fmaf(s[c], prm.scale_log2, neg_m);
+                    const float x1 = fmaf(s[c + 1], prm.scale_log2, neg_m);
+                    float p0, p1;
+                    if (!ragged && (c & 6) == 6) {           // 1 pair in 4 on the FMA pipe
+                        p0 = ex2_poly(x0);
+                        p1 = ex2_poly(x1);
+                    } else {
+                        p0 = ex2_mufu(x0);
+                        p1 = ex2_mufu(x1);
+                    }
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[c / 2] = pack_bf16(p0, p1);
                 }
-                l = l * alpha + rowsum;
-                // the previous PV must be done before P is overwritten and O is touched
+                l = l * alpha + (sum0 + sum1);
+                // P_j (bf16 pairs) into P buffer j%2; its previous reader, PV(kv_it-2),
+                // completed before the S_FULL commit waited on above.
+                const uint32_t p_addr = tmem + lane_base + (sb ? kColP1 : kColP0) + half * (HC / 2);
+                if constexpr (HC / 2 == 32) {
+                    tmem_st32(p_addr, pk);
+                } else {
+                    tmem_st16(p_addr, pk);
+                }
+                // the previous PV must be done before O is rescaled; waiting on it every
+                // block keeps at most one PV completion outstanding for this warp
                 if (local > 0) {
                     if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
                     ++pv_it;
                     tc_fence_after();
-                }
-                // P row -> swizzled smem slab(s): 16-byte chunk u of row `row` lands at
-                // chunk u ^ (row % 8) inside the row's 128-byte line
-                unsigned char* prow = smem + L::offP + (row / 8) * 1024 + (row % 8) * 128;
+                    if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                for (int u = 0; u < BLK / 8; ++u) {
-                    const int slab = u / 8, cu = u % 8;
-                    uint4 v = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
-                    *reinterpret_cast<uint4*>(prow + slab * kTileM * 128 + ((cu ^ (row % 8)) * 16)) = v;
-                }
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const float a = rescale ? alpha : 1.f;
+                        for (int c = 0; c < OC / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tmem + lane_base + kColO + half * OC + c * 32, o);
+                            tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + kColO + c * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
-                        tmem_st32(tmem + lane_base + kColO + c * 32, o);
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st32(tmem + lane_base + kColO + half * OC + c * 32, o);
+                        }
                     }
-                    tmem_wait_st();
                 }
-                fence_proxy_async();
+                tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(B_PFULL));
                 ++kv_it;
                 ++local;
             }
             if (!ok) break;
-            // epilogue: last PV of the item, then O / l to the token's raster position
+            // epilogue: last PV of the item; the two partial row sums meet in shared
+            // memory (slots alternate by item; a bounded mbarrier pairs the two warps)
             if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
             ++pv_it;
             tc_fence_after();
-            const float inv = 1.f / l;
-            __nv_bfloat16* dst = prm.o + (((int64_t)b * prm.N + (row_real ? prm.perm[n_tok] : 0)) * prm.H + h) * D;
+            float* ls = xchg + (items & 1) * 2 * kTileM;
+            ls[half * kTileM + row] = l;
+            mbar_arrive(bar(B_PAIR0 + quad));
+            if (!(ok = warp_wait(bar(B_PAIR0 + quad), items & 1, abort_flag))) break;
+            ++items;
+            const float inv = 1.f / (l + ls[(1 - half) * kTileM + row]);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < OC / 32; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tmem + lane_base + kColO + c * 32, o);
+                tmem_ld32(tmem + lane_base + kColO + half * OC + c * 32, o);
                 tmem_wait_ld();
                 if (row_real) {
 #pragma unroll
