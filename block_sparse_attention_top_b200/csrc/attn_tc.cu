@@ -6,14 +6,16 @@
 // (one item = one 128-row query tile of one head).  Per item and retained key
 // block j, with S, P and O living in tensor memory (TMEM):
 //
-//   warp 0 (1 thread)   TMA: Q tile once per item; K_j, V_j into 2-stage rings
+//   warp 0 (1 thread)   TMA: Q tile once per item; K_j into a 3-stage ring
+//   warp 10 (1 thread)  TMA: V_j into a 2-stage ring (runs ahead independently of K)
 //   warp 1 (1 thread)   tcgen05.mma: S[j%2] = Q K_j^T      (M=128, N=block, K=d; A, B in smem)
 //                                    O     += P[j%2] V_j   (M=128, N=d, K=block; P in TMEM)
 //   warps 2..9          softmax: TMEM lane = query row; each row is split over
 //                       two warps, one per half of the key (and output)
-//                       columns.  Both read the whole S row for its maximum, so
-//                       no exchange is needed per block.  Online softmax in the
-//                       log2 domain; a quarter of the exponentials run as a
+//                       columns, which swap their half-row maxima (and at the
+//                       end their row sums) through shared memory behind a
+//                       bounded per-quadrant mbarrier.  Online softmax in the
+//                       log2 domain; one exponential in eight runs as a
 //                       polynomial on the FMA pipe to offload the MUFU unit;
 //                       P_j goes to its own TMEM columns as bf16 pairs
 //                       (tcgen05.st); the O row is rescaled in TMEM only when
@@ -26,7 +28,8 @@
 // on the tensor pipe while the softmax warps work on block j.  TMEM columns:
 // S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
 //
-// Every wait on an mbarrier is bounded (about 4 s of %globaltimer); on expiry
+// Every wait on an mbarrier spins on test_wait and is bounded (about 4 s of
+// %globaltimer, checked every 1024 probes); on expiry
 // the CTA records BSA_EDEVICE, raises a shared abort flag that stops the other
 // roles, drains its own tensor-core work and frees TMEM before returning.
 #include <cuda.h>
@@ -41,7 +44,9 @@ namespace bsa {
 namespace {
 
 constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = 32 * (2 + kSoftmaxWarps);   // producer, MMA, softmax
+constexpr int kThreads = 32 * (3 + kSoftmaxWarps);   // Q/K producer, MMA, softmax x8, V producer
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kVWarp = 2 + kSoftmaxWarps;
 constexpr int kTileM = 128;                          // query rows per tile (TMEM lanes)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
@@ -65,28 +70,33 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Non-blocking probe of a phase.  The suspending try_wait form was measured to
+// wake up late (about 1000 cycles after the phase completed), which sat on
+// the critical path of every handshake; the waits below spin on test_wait.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false if the abort flag is raised or the time limit passes.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
     const unsigned long long t0 = globaltimer();
     for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 63u) == 0) {
+        if (mbar_test(bar, parity)) return true;
+        if ((n & 1023u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer() - t0 > kTimeoutNs) return false;
         }
     }
+}
+// Bounded wait: false if the abort flag is raised or the time limit passes.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, abort_flag);
 }
 // Warp-uniform bounded wait (every lane polls; all lanes agree on the outcome).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -192,21 +202,79 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
-// 2^x on the FMA pipe for x in [-127, 128): split x = j + f with j = rint(x),
+
+// Packed fp32 pairs (sm_100 f32x2 instructions): d = a * b + c, d = a + b.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// 2^x for a pair of values on the FMA pipe for x in [-127, 128): split x = j + f with j = rint(x),
 // f in [-1/2, 1/2] (adding 1.5 * 2^23 rounds to an integer held in the low
 // mantissa bits), a degree-3 polynomial for 2^f (coefficients from a
 // relative-error minimax fit on [-1/2, 1/2], max relative error 7.5e-5), and
 // j added straight into the exponent field.  Accurate far beyond the bf16
 // rounding P receives.
-__device__ __forceinline__ float ex2_poly(float x) {
-    x = fmaxf(x, -127.f);
-    const float t = x + 12582912.f;
-    const float j = t - 12582912.f;
-    const float f = x - j;
-    float p = fmaf(0.0551716648f, f, 0.2426111251f);
-    p = fmaf(p, f, 0.6932609677f);
-    p = fmaf(p, f, 0.9999280572f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
+    x0 = fmaxf(x0, -127.f);
+    x1 = fmaxf(x1, -127.f);
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    fadd2(t0, t1, x0, x1, 12582912.f, 12582912.f);
+    fadd2(j0, j1, t0, t1, -12582912.f, -12582912.f);
+    ffma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);
+    ffma2(p0, p1, 0.0551716648f, 0.0551716648f, f0, f1, 0.2426111251f, 0.2426111251f);
+    ffma2(p0, p1, p0, p1, f0, f1, 0.6932609677f, 0.6932609677f);
+    ffma2(p0, p1, p0, p1, f0, f1, 0.9999280572f, 0.9999280572f);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Maximum of n values with 8 independent chains (n a multiple of 16).
+template <int n>
+__device__ __forceinline__ float row_max(const uint32_t* v, float init) {
+    float m[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) m[u] = max3(init, __uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]));
+#pragma unroll
+    for (int c = 16; c < n; c += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m[u] = max3(m[u], __uint_as_float(v[c + 2 * u]), __uint_as_float(v[c + 2 * u + 1]));
+    return fmaxf(fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5])), fmaxf(m[6], m[7]));
+}
+
+// P for this warp's half row: p = 2^(s * scale - m), packed to bf16 pairs, and
+// the half-row sum.  One pair in eight goes through the FMA-pipe polynomial
+// unless the block is ragged (masked keys are -inf there).
+template <int HC, bool RAGGED>
+__device__ __forceinline__ float softmax_half(const uint32_t* s, float scale, float neg_m, uint32_t* pk) {
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+#pragma unroll
+    for (int c = 0; c < HC; c += 2) {
+        float x0, x1, p0, p1;
+        ffma2(x0, x1, __uint_as_float(s[c]), __uint_as_float(s[c + 1]), scale, scale, neg_m, neg_m);
+        if (!RAGGED && (c & 14) == 14) {
+            ex2_poly2(x0, x1, p0, p1);
+        } else {
+            p0 = ex2_mufu(x0);
+            p1 = ex2_mufu(x1);
+        }
+        const int u = (c / 2) & 3;
+        fadd2(acc[2 * u], acc[2 * u + 1], acc[2 * u], acc[2 * u + 1], p0, p1);
+        pk[c / 2] = pack_bf16(p0, p1);
+    }
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 // ------------------------------------------------------------- shared layout
@@ -216,18 +284,19 @@ struct Smem {
     static constexpr int kKV = BLK * D * 2;         // one K or V tile: D/64 slabs of [BLK rows x 128 B]
     static constexpr int offQ = 0;
     static constexpr int offK = offQ + kQ;
-    static constexpr int offV = offK + 2 * kKV;
-    static constexpr int offXchg = offV + 2 * kKV;  // float [2 item parity][2 half][128 rows] row sums
-    static constexpr int offBar = offXchg + 2 * 2 * kTileM * 4;
-    static constexpr int kBars = 20;
+    static constexpr int offV = offK + kKStages * kKV;
+    // float [2 kv parity][2 half][128 rows] half-row maxima, then the same for row sums by item parity
+    static constexpr int offXchg = offV + kVStages * kKV;
+    static constexpr int offBar = offXchg + 2 * 2 * 2 * kTileM * 4;
+    static constexpr int kBars = 24;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kBytes = offMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;   // room to align the base to 1024 B
 };
 // barrier slots
-enum { B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0,
-       B_VEMPTY1, B_SFULL0, B_SFULL1, B_PFULL, B_PVDONE, B_DRAIN, B_PAIR0, B_PAIR1, B_PAIR2, B_PAIR3,
-       B_COUNT };
+enum { B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KEMPTY0 = B_KFULL0 + kKStages, B_VFULL0 = B_KEMPTY0 + kKStages,
+       B_VEMPTY0 = B_VFULL0 + kVStages, B_SFULL0 = B_VEMPTY0 + kVStages, B_SFULL1, B_PFULL, B_PVDONE, B_DRAIN,
+       B_PAIR0, B_PAIR1, B_PAIR2, B_PAIR3, B_COUNT };
 
 struct Params {
     const int32_t* row_ptr;
@@ -293,8 +362,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int grid = gridDim.x, cta = blockIdx.x;
     const int nb = prm.nb;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == kVWarp) {
+        // ------------------------------------------------------------ producers
+        // warp 0: Q once per item and the K ring; warp kVWarp: the V ring.  Both
+        // walk the same item and column sequence, so their ring indices agree
+        // with the MMA thread's.
+        const bool kside = warp == 0;
         if (lane == 0) {
             uint32_t kv_it = 0, q_it = 0;
             bool ok = true;
@@ -307,29 +380,38 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 for (int jj = beg; jj < end; ++jj) nvalid += valid_col(prm.col_idx[jj], nb);
                 if (nvalid == 0) continue;
                 const int bh = r / nb, i = r % nb;
-                if (q_it > 0 && !(ok = mbar_wait(bar(B_QEMPTY), (q_it - 1) & 1, abort_flag))) break;
-                mbar_expect_tx(bar(B_QFULL), BLK * D * 2);
-                for (int s = 0; s < D / 64; ++s)
-                    tma_load_2d(sbase + L::offQ + s * kTileM * 128, &tmQ, s * 64,
-                                (int)(bh * prm.npad + (int64_t)i * BLK), bar(B_QFULL));
-                ++q_it;
+                if (kside) {
+                    if (q_it > 0 && !(ok = mbar_wait(bar(B_QEMPTY), (q_it - 1) & 1, abort_flag))) break;
+                    mbar_expect_tx(bar(B_QFULL), BLK * D * 2);
+                    for (int s = 0; s < D / 64; ++s)
+                        tma_load_2d(sbase + L::offQ + s * kTileM * 128, &tmQ, s * 64,
+                                    (int)(bh * prm.npad + (int64_t)i * BLK), bar(B_QFULL));
+                    ++q_it;
+                }
                 for (int jj = beg; jj < end; ++jj) {
                     const int j = prm.col_idx[jj];
                     if (!valid_col(j, nb)) {
-                        record_error(prm.err, BSA_EDEVICE, r);
+                        if (kside) record_error(prm.err, BSA_EDEVICE, r);
                         continue;
                     }
-                    const int st = kv_it & 1;
-                    const uint32_t ph = ((kv_it >> 1) & 1) ^ 1;
                     const int y = (int)(bh * prm.npad + (int64_t)j * BLK);
-                    if (kv_it >= 2 && !(ok = mbar_wait(bar(B_KEMPTY0 + st), ph, abort_flag))) break;
-                    mbar_expect_tx(bar(B_KFULL0 + st), L::kKV);
-                    for (int s = 0; s < D / 64; ++s)
-                        tma_load_2d(sbase + L::offK + st * L::kKV + s * BLK * 128, &tmK, s * 64, y, bar(B_KFULL0 + st));
-                    if (kv_it >= 2 && !(ok = mbar_wait(bar(B_VEMPTY0 + st), ph, abort_flag))) break;
-                    mbar_expect_tx(bar(B_VFULL0 + st), L::kKV);
-                    for (int s = 0; s < D / 64; ++s)
-                        tma_load_2d(sbase + L::offV + st * L::kKV + s * BLK * 128, &tmV, s * 64, y, bar(B_VFULL0 + st));
+                    if (kside) {
+                        const int st = kv_it % kKStages;
+                        const uint32_t use = kv_it / kKStages;
+                        if (use > 0 && !(ok = mbar_wait(bar(B_KEMPTY0 + st), (use - 1) & 1, abort_flag))) break;
+                        mbar_expect_tx(bar(B_KFULL0 + st), L::kKV);
+                        for (int s = 0; s < D / 64; ++s)
+                            tma_load_2d(sbase + L::offK + st * L::kKV + s * BLK * 128, &tmK, s * 64, y,
+                                        bar(B_KFULL0 + st));
+                    } else {
+                        const int st = kv_it % kVStages;
+                        const uint32_t use = kv_it / kVStages;
+                        if (use > 0 && !(ok = mbar_wait(bar(B_VEMPTY0 + st), (use - 1) & 1, abort_flag))) break;
+                        mbar_expect_tx(bar(B_VFULL0 + st), L::kKV);
+                        for (int s = 0; s < D / 64; ++s)
+                            tma_load_2d(sbase + L::offV + st * L::kKV + s * BLK * 128, &tmV, s * 64, y,
+                                        bar(B_VFULL0 + st));
+                    }
                     ++kv_it;
                 }
             }
@@ -345,8 +427,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             // O += P V for kv iteration `it`; P sits in TMEM buffer it&1
             auto issue_pv = [&](uint32_t it, bool first) -> bool {
                 if (!mbar_wait(bar(B_PFULL), pv_it & 1, abort_flag)) return false;
-                const int st = it & 1;
-                if (!mbar_wait(bar(B_VFULL0 + st), (it >> 1) & 1, abort_flag)) return false;
+                const int st = it % kVStages;
+                if (!mbar_wait(bar(B_VFULL0 + st), (it / kVStages) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t p_tmem = tmem + ((it & 1) ? kColP1 : kColP0);
 #pragma unroll
@@ -372,10 +454,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 int local = 0;
                 for (int jj = beg; jj < end && ok; ++jj) {
                     if (!valid_col(prm.col_idx[jj], nb)) continue;
-                    const int st = kv_it & 1;
+                    const int st = kv_it % kKStages;
                     // S buffer kv_it&1 is free: the softmax warps read S(kv_it-2) before the
                     // P_FULL arrival that this thread waited on for PV(kv_it-2).
-                    if (!(ok = mbar_wait(bar(B_KFULL0 + st), (kv_it >> 1) & 1, abort_flag))) break;
+                    if (!(ok = mbar_wait(bar(B_KFULL0 + st), (kv_it / kKStages) & 1, abort_flag))) break;
                     tc_fence_after();
                     const uint32_t d_s = tmem + ((kv_it & 1) ? kColS1 : kColS0);
 #pragma unroll
@@ -408,7 +490,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int half = (warp - 2) >> 2;                // which half of the key / output columns
         const int row = 32 * quad + lane;                // TMEM lane == query row in tile
         const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-        uint32_t kv_it = 0, pv_it = 0, items = 0;
+        uint32_t kv_it = 0, pv_it = 0, items = 0, pairs = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int idx = item_index(k, cta, grid);
@@ -440,45 +522,24 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // padding keys of a ragged last block
                 const int valid_keys = prm.N - j * BLK;
                 const bool ragged = valid_keys < BLK;
-                float s[HC];
-                float lm0, lm1;
-                {
-                    // the other half: only its maximum is needed
-                    uint32_t raw[HC];
+                uint32_t sv[HC];                          // this warp's half of the S row
 #pragma unroll
-                    for (int c = 0; c < HC / 32; ++c)
-                        tmem_ld32(tmem + lane_base + s_col + (1 - half) * HC + c * 32, raw + 32 * c);
-                    tmem_wait_ld();
-                    if (ragged) {
-#pragma unroll
-                        for (int c = 0; c < HC; ++c)
-                            if ((1 - half) * HC + c >= valid_keys) raw[c] = __float_as_uint(-INFINITY);
-                    }
-                    lm0 = __uint_as_float(raw[0]);
-                    lm1 = __uint_as_float(raw[1]);
-#pragma unroll
-                    for (int c = 2; c + 1 < HC; c += 4) {
-                        lm0 = max3(lm0, __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
-                        if (c + 3 < HC) lm1 = max3(lm1, __uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3]));
-                    }
-#pragma unroll
-                    for (int c = 0; c < HC / 32; ++c)
-                        tmem_ld32(tmem + lane_base + s_col + half * HC + c * 32, raw + 32 * c);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < HC; ++c) s[c] = __uint_as_float(raw[c]);
-                }
+                for (int c = 0; c < HC / 32; ++c) tmem_ld32(tmem + lane_base + s_col + half * HC + c * 32, sv + 32 * c);
+                tmem_wait_ld();
                 if (ragged) {
 #pragma unroll
                     for (int c = 0; c < HC; ++c)
-                        if (half * HC + c >= valid_keys) s[c] = -INFINITY;
+                        if (half * HC + c >= valid_keys) sv[c] = __float_as_uint(-INFINITY);
                 }
-#pragma unroll
-                for (int c = 0; c + 1 < HC; c += 4) {
-                    lm0 = max3(lm0, s[c], s[c + 1]);
-                    if (c + 3 < HC) lm1 = max3(lm1, s[c + 2], s[c + 3]);
-                }
-                const float mx = fmaxf(lm0, lm1) * prm.scale_log2;
+                // the two half-row maxima meet in shared memory (slots alternate with
+                // the kv parity; the pair mbarrier completes once per block)
+                const float lmax = row_max<HC>(sv, -INFINITY);
+                float* xs = xchg + sb * 2 * kTileM;
+                xs[half * kTileM + row] = lmax;
+                mbar_arrive(bar(B_PAIR0 + quad));
+                if (!(ok = warp_wait(bar(B_PAIR0 + quad), pairs & 1, abort_flag))) break;
+                ++pairs;
+                const float mx = fmaxf(lmax, xs[(1 - half) * kTileM + row]) * prm.scale_log2;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (local == 0) {
@@ -488,26 +549,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     m_use = mx;
                     rescale = true;
                 }
-                const float neg_m = -m_use;
-                float sum0 = 0.f, sum1 = 0.f;
                 uint32_t pk[HC / 2];
-#pragma unroll
-                for (int c = 0; c < HC; c += 2) {
-                    const float x0 = fmaf(s[c], prm.scale_log2, neg_m);
-                    const float x1 = fmaf(s[c + 1], prm.scale_log2, neg_m);
-                    float p0, p1;
-                    if (!ragged && (c & 6) == 6) {           // 1 pair in 4 on the FMA pipe
-                        p0 = ex2_poly(x0);
-                        p1 = ex2_poly(x1);
-                    } else {
-                        p0 = ex2_mufu(x0);
-                        p1 = ex2_mufu(x1);
-                    }
-                    sum0 += p0;
-                    sum1 += p1;
-                    pk[c / 2] = pack_bf16(p0, p1);
-                }
-                l = l * alpha + (sum0 + sum1);
+                const float rowsum = ragged ? softmax_half<HC, true>(sv, prm.scale_log2, -m_use, pk)
+                                            : softmax_half<HC, false>(sv, prm.scale_log2, -m_use, pk);
+                l = l * alpha + rowsum;
                 // P_j (bf16 pairs) into P buffer j%2; its previous reader, PV(kv_it-2),
                 // completed before the S_FULL commit waited on above.
                 const uint32_t p_addr = tmem + lane_base + (sb ? kColP1 : kColP0) + half * (HC / 2);
@@ -546,10 +591,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
             ++pv_it;
             tc_fence_after();
-            float* ls = xchg + (items & 1) * 2 * kTileM;
+            float* ls = xchg + 4 * kTileM + (items & 1) * 2 * kTileM;
             ls[half * kTileM + row] = l;
             mbar_arrive(bar(B_PAIR0 + quad));
-            if (!(ok = warp_wait(bar(B_PAIR0 + quad), items & 1, abort_flag))) break;
+            if (!(ok = warp_wait(bar(B_PAIR0 + quad), pairs & 1, abort_flag))) break;
+            ++pairs;
             ++items;
             const float inv = 1.f / (l + ls[(1 - half) * kTileM + row]);
 #pragma unroll

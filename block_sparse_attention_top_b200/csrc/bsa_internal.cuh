@@ -5,7 +5,7 @@
 #include <stdint.h>
 #include <stddef.h>
 
-#include "../../include/bsa.h"
+#include "bsa.h"
 
 struct bsa_plan {
     int B, H, T, Hs, Ws, d, block, order;
