@@ -16,11 +16,15 @@ import os
 
 import torch
 
-_HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libbsa.so")
+from . import build as _build
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libbsa.so not built at {LIB_PATH}: run `python -m block_sparse_attention_top_b200.build`")
+LIB_PATH = _build.LIB
+if _build.stale():
+    # missing or older than its sources: build it now, or fail loudly (there is no CPU path)
+    try:
+        _build.build()
+    except Exception as exc:  # noqa: BLE001
+        raise ImportError(f"libbsa.so at {LIB_PATH} is missing or stale and could not be built: {exc}") from exc
 _lib = ctypes.CDLL(LIB_PATH)
 
 BSA_OK, BSA_EINVAL, BSA_EUNSUPPORTED, BSA_ECAPACITY, BSA_EWORKSPACE, BSA_ECUDA, BSA_EDEVICE = 0, -1, -2, -3, -4, -5, -6

@@ -28,7 +28,8 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
+def stale() -> bool:
+    """True if libbsa.so is missing or older than any source it is built from."""
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
@@ -37,7 +38,7 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+    if not force and not stale():
         return LIB
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
