@@ -44,6 +44,7 @@ _SIGS = {
     "bsa_token_order": (_I, [_I, _I, _I, _I, _P]),
     "bsa_workspace_size": (_SZ, [_P, _I]),
     "bsa_route": (_I, [_P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
+    "bsa_route_static": (_I, [_P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _I64, _P, _P, _P]),
     "bsa_route_intermediates": (_I, [_P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P)]),
     "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -130,6 +131,13 @@ def bsa_route(plan, q, k, dtype, p, k_floor, row_ptr, col_idx, col_cap, L_h, nnz
     return _lib.bsa_route(plan.handle, _ptr(q), _ptr(k), dtype, float(p), int(k_floor), _ptr(row_ptr),
                           _ptr(col_idx), int(col_cap), _ptr(L_h), _ptr(nnz), _ptr(workspace),
                           workspace.numel() if workspace is not None else 0, _stream(stream))
+
+
+def bsa_route_static(plan, q, k, dtype, p, k_floor, row_ptr, col_idx, col_cap, L_h, nnz, stream=None):
+    """bsa_route with the library's fixed device scratch instead of a caller workspace
+    (for callers that cannot allocate when they route)."""
+    return _lib.bsa_route_static(plan.handle, _ptr(q), _ptr(k), dtype, float(p), int(k_floor), _ptr(row_ptr),
+                                 _ptr(col_idx), int(col_cap), _ptr(L_h), _ptr(nnz), _stream(stream))
 
 
 def bsa_route_intermediates(plan, workspace):
