@@ -376,9 +376,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (idx >= prm.rows) break;
                 const int r = prm.work[idx];
                 const int beg = prm.row_ptr[r], end = prm.row_ptr[r + 1];
-                int nvalid = 0;
-                for (int jj = beg; jj < end; ++jj) nvalid += valid_col(prm.col_idx[jj], nb);
-                if (nvalid == 0) continue;
+                if (end <= beg) continue;                    // no key block: no Q either
                 const int bh = r / nb, i = r % nb;
                 if (kside) {
                     if (q_it > 0 && !(ok = mbar_wait(bar(B_QEMPTY), (q_it - 1) & 1, abort_flag))) break;
@@ -388,8 +386,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                     (int)(bh * prm.npad + (int64_t)i * BLK), bar(B_QFULL));
                     ++q_it;
                 }
+                int jn = prm.col_idx[beg];
                 for (int jj = beg; jj < end; ++jj) {
-                    const int j = prm.col_idx[jj];
+                    const int j = jn;
+                    if (jj + 1 < end) jn = prm.col_idx[jj + 1];   // next column, one iteration ahead
                     if (!valid_col(j, nb)) {
                         if (kside) record_error(prm.err, BSA_EDEVICE, r);
                         continue;
@@ -446,14 +446,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (idx >= prm.rows) break;
                 const int r = prm.work[idx];
                 const int beg = prm.row_ptr[r], end = prm.row_ptr[r + 1];
-                int nvalid = 0;
-                for (int jj = beg; jj < end; ++jj) nvalid += valid_col(prm.col_idx[jj], nb);
-                if (nvalid == 0) continue;
+                if (end <= beg) continue;
                 if (!(ok = mbar_wait(bar(B_QFULL), q_it & 1, abort_flag))) break;
                 ++q_it;
                 int local = 0;
+                bool q_released = false;
+                int jn = prm.col_idx[beg];
                 for (int jj = beg; jj < end && ok; ++jj) {
-                    if (!valid_col(prm.col_idx[jj], nb)) continue;
+                    const int j = jn;
+                    if (jj + 1 < end) jn = prm.col_idx[jj + 1];   // next column, one iteration ahead
+                    if (!valid_col(j, nb)) continue;
                     const int st = kv_it % kKStages;
                     // S buffer kv_it&1 is free: the softmax warps read S(kv_it-2) before the
                     // P_FULL arrival that this thread waited on for PV(kv_it-2).
@@ -468,12 +470,17 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                     tc_commit(bar(B_SFULL0 + (kv_it & 1)));
                     tc_commit(bar(B_KEMPTY0 + st));
-                    if (local == nvalid - 1) tc_commit(bar(B_QEMPTY));
+                    if (jj == end - 1) {                           // last QK of the item: Q may be replaced
+                        tc_commit(bar(B_QEMPTY));
+                        q_released = true;
+                    }
                     if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
                     ++kv_it;
                     ++local;
                 }
-                if (ok && !(ok = issue_pv(kv_it - 1, nvalid == 1))) break;
+                if (!ok) break;
+                if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
+                if (!q_released) tc_commit(bar(B_QEMPTY));         // trailing invalid columns
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -497,23 +504,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             if (idx >= prm.rows) break;
             const int r = prm.work[idx];
             const int beg = prm.row_ptr[r], end = prm.row_ptr[r + 1];
-            int nvalid = 0;
-            for (int jj = beg; jj < end; ++jj) nvalid += valid_col(prm.col_idx[jj], nb);
             const int bh = r / nb, i = r % nb;
             const int b = bh / prm.H, h = bh % prm.H;
             const int n_tok = i * BLK + row;             // reordered position of this row
             const bool row_real = row < BLK && n_tok < prm.N;
             __nv_bfloat16* dst = prm.o + (((int64_t)b * prm.N + (row_real ? prm.perm[n_tok] : 0)) * prm.H + h) * D +
                                  half * OC;
-            if (nvalid == 0) {
-                if (row_real)
-                    for (int c = 0; c < OC / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
-                continue;
-            }
             float m_use = 0.f, l = 0.f;
             int local = 0;
+            int jn = end > beg ? prm.col_idx[beg] : 0;
             for (int jj = beg; jj < end && ok; ++jj) {
-                const int j = prm.col_idx[jj];
+                const int j = jn;
+                if (jj + 1 < end) jn = prm.col_idx[jj + 1];   // next column, one iteration ahead
                 if (!valid_col(j, nb)) continue;
                 const int sb = kv_it & 1;
                 const uint32_t s_col = sb ? kColS1 : kColS0;
@@ -586,6 +588,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 ++local;
             }
             if (!ok) break;
+            if (local == 0) {                            // no (valid) key block: zeros
+                if (row_real)
+                    for (int c = 0; c < OC / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+                continue;
+            }
             // epilogue: last PV of the item; the two partial row sums meet in shared
             // memory (slots alternate by item; a bounded mbarrier pairs the two warps)
             if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
