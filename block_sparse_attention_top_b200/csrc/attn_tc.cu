@@ -8,8 +8,9 @@
 //
 //   warp 0 (1 thread)   TMA: Q tile once per item; K_j into a 3-stage ring
 //   warp 10 (1 thread)  TMA: V_j into a 2-stage ring (runs ahead independently of K)
-//   warp 1 (1 thread)   tcgen05.mma: S[j%2] = Q K_j^T      (M=128, N=block, K=d; A, B in smem)
-//                                    O     += P[j%2] V_j   (M=128, N=d, K=block; P in TMEM)
+//   warp 1 (1 thread)   tcgen05.cp: Q tile smem -> TMEM once per item;
+//                       tcgen05.mma: S[j%2] = Q K_j^T   (M=128, N=block, K=d; Q in TMEM, K in smem)
+//                                    O     += P_j V_j   (M=128, N=d, K=block; P in TMEM, V in smem)
 //   warps 2..9          softmax: TMEM lane = query row; each row is split over
 //                       two warps, one per half of the key (and output)
 //                       columns, which swap their half-row maxima (and at the
@@ -17,16 +18,18 @@
 //                       bounded per-quadrant mbarrier.  Online softmax in the
 //                       log2 domain; one exponential in eight runs as a
 //                       polynomial on the FMA pipe to offload the MUFU unit;
-//                       P_j goes to its own TMEM columns as bf16 pairs
-//                       (tcgen05.st); the O row is rescaled in TMEM only when
+//                       P_j overwrites the first half of S_j's TMEM columns as
+//                       bf16 pairs (tcgen05.st); the O row is rescaled in TMEM only when
 //                       its running max grows by more than 2^8.  Epilogue: the
 //                       two partial row sums meet through shared memory, then
 //                       O / l, bf16, stored at the token's raster position (the
 //                       inverse Hilbert permutation is fused into this store).
 //
-// S and P are double-buffered, so QK^T of block j+1 and PV of block j-1 run
-// on the tensor pipe while the softmax warps work on block j.  TMEM columns:
-// S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+// S (with P) is double-buffered, so QK^T of block j+1 and PV of block j-1 run
+// on the tensor pipe while the softmax warps work on block j.  Keeping Q in
+// TMEM halves the shared-memory reads of QK^T, which would otherwise need the
+// SM's whole shared-memory bandwidth at full MMA rate.  TMEM columns:
+// S0 [0,128) S1 [128,256) O [256,384) Q [384,448).
 //
 // Every wait on an mbarrier spins on test_wait and is bounded (about 4 s of
 // %globaltimer, checked every 1024 probes); on expiry
@@ -49,7 +52,7 @@ constexpr int kKStages = 3, kVStages = 2;
 constexpr int kVWarp = 2 + kSoftmaxWarps;
 constexpr int kTileM = 128;                          // query rows per tile (TMEM lanes)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColQ = 384;
 constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
 // ---------------------------------------------------------------- PTX helpers
@@ -121,15 +124,9 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+// 128 rows x 256 bits from shared memory (matrix descriptor) into TMEM lanes 0..127
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
 }
 // D[tmem] (+)= A[tmem] * B[smem desc]
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -430,7 +427,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const int st = it % kVStages;
                 if (!mbar_wait(bar(B_VFULL0 + st), (it / kVStages) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t p_tmem = tmem + ((it & 1) ? kColP1 : kColP0);
+                const uint32_t p_tmem = tmem + ((it & 1) ? kColS1 : kColS0);   // P overwrote S(it)
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
                     const uint64_t b = smem_desc(sbase + L::offV + st * L::kKV + kk * 16 * 128, BLK * 128, 1024);
@@ -449,8 +446,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (end <= beg) continue;
                 if (!(ok = mbar_wait(bar(B_QFULL), q_it & 1, abort_flag))) break;
                 ++q_it;
+                // Q -> TMEM (16 columns of bf16 per copy), then its shared buffer is free.
+                // The previous item's QKs, issued earlier by this thread, have read the
+                // old Q columns: tensor-core operations of one thread run in issue order.
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc_cp_128x256b(tmem + kColQ + kk * 8,
+                                   smem_desc(sbase + L::offQ + (kk / 4) * kTileM * 128 + (kk % 4) * 32, 16, 1024));
+                tc_commit(bar(B_QEMPTY));
                 int local = 0;
-                bool q_released = false;
                 int jn = prm.col_idx[beg];
                 for (int jj = beg; jj < end && ok; ++jj) {
                     const int j = jn;
@@ -458,29 +463,24 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     if (!valid_col(j, nb)) continue;
                     const int st = kv_it % kKStages;
                     // S buffer kv_it&1 is free: the softmax warps read S(kv_it-2) before the
-                    // P_FULL arrival that this thread waited on for PV(kv_it-2).
+                    // P_FULL arrival this thread waited on for PV(kv_it-2), and that PV, which
+                    // read P from the same columns, was issued earlier by this thread.
                     if (!(ok = mbar_wait(bar(B_KFULL0 + st), (kv_it / kKStages) & 1, abort_flag))) break;
                     tc_fence_after();
                     const uint32_t d_s = tmem + ((kv_it & 1) ? kColS1 : kColS0);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t a = smem_desc(sbase + L::offQ + (kk / 4) * kTileM * 128 + (kk % 4) * 32, 16, 1024);
                         const uint64_t b = smem_desc(sbase + L::offK + st * L::kKV + (kk / 4) * BLK * 128 + (kk % 4) * 32, 16, 1024);
-                        tc_mma_ss(d_s, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                        tc_mma_ts(d_s, tmem + kColQ + kk * 8, b, idesc_qk, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(bar(B_SFULL0 + (kv_it & 1)));
                     tc_commit(bar(B_KEMPTY0 + st));
-                    if (jj == end - 1) {                           // last QK of the item: Q may be replaced
-                        tc_commit(bar(B_QEMPTY));
-                        q_released = true;
-                    }
                     if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
                     ++kv_it;
                     ++local;
                 }
                 if (!ok) break;
                 if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
-                if (!q_released) tc_commit(bar(B_QEMPTY));         // trailing invalid columns
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -555,9 +555,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const float rowsum = ragged ? softmax_half<HC, true>(sv, prm.scale_log2, -m_use, pk)
                                             : softmax_half<HC, false>(sv, prm.scale_log2, -m_use, pk);
                 l = l * alpha + rowsum;
-                // P_j (bf16 pairs) into P buffer j%2; its previous reader, PV(kv_it-2),
-                // completed before the S_FULL commit waited on above.
-                const uint32_t p_addr = tmem + lane_base + (sb ? kColP1 : kColP0) + half * (HC / 2);
+                // P_j (bf16 pairs) over the first half of S_j's columns: both warps of the
+                // pair read their S halves before the exchange above.
+                const uint32_t p_addr = tmem + lane_base + s_col + half * (HC / 2);
                 if constexpr (HC / 2 == 32) {
                     tmem_st32(p_addr, pk);
                 } else {
