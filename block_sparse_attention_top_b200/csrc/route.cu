@@ -3,9 +3,10 @@
 // a Top-k safety floor; L_h from the review's Eq. 1).
 //
 //   k_pool       gather through the token order + block mean of Q and K (HBM bound)
-//   k_scores     s_ij = <Qbar_i, Kbar_j> / sqrt(d), fp64 tiles
-//   k_route_rows softmax, sort by (P desc, j asc), cumulative mass, Top-p cut,
-//                Top-k floor -> count and importance order per row
+//   k_scores     s_ij = <Qbar_i, Kbar_j> / sqrt(d), register-tiled fp64
+//   k_route_warp softmax, sort by (P desc, j asc), cumulative mass, Top-p cut,
+//   k_route_cta  Top-k floor -> count and importance order per row (one warp
+//                per row up to 256 blocks, one CTA per row above)
 //   k_csr_scan   exclusive scan of the counts -> row_ptr, nnz, L_h
 //   k_csr_fill   copy each row's kept columns into col_idx
 //
@@ -26,7 +27,7 @@ namespace {
 // (one 16-byte load per token) and sums them over the block's tokens.
 // ---------------------------------------------------------------------------
 constexpr int kPoolThreads = 256;
-constexpr int kPoolUnroll = 8;
+constexpr int kPoolUnroll = 16;
 
 template <typename T> struct Vec16;
 template <> struct Vec16<__nv_bfloat16> {
@@ -104,48 +105,78 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Scores: 64x64 output tile per CTA, 256 threads x (4x4) outputs, fp64 FMA,
-// d consumed in slices of 16 through shared memory.
+// Scores: TM x TM output tile per CTA (TM = 64 or 128), 256 threads, each
+// (TM/16) x (TM/16) outputs held in registers; d consumed in slices of 16
+// staged through shared memory; fp64 FMA.
 // ---------------------------------------------------------------------------
-constexpr int kST = 64, kSK = 16;
+constexpr int kSK = 16;
 
+template <int TM>
 __global__ void __launch_bounds__(256)
 k_scores(const double* __restrict__ qbar, const double* __restrict__ kbar, double* __restrict__ S,
          int nb, int d, double scale) {
-    __shared__ double As[kSK][kST + 1];
-    __shared__ double Bs[kSK][kST + 1];
+    constexpr int R = TM / 16;
+    constexpr int L = TM * kSK / 256;                 // elements of each operand loaded per thread per slice
+    extern __shared__ double score_smem[];             // [2 operands][2 buffers][kSK][TM + 1]
+    auto As = reinterpret_cast<double (*)[kSK][TM + 1]>(score_smem);
+    auto Bs = reinterpret_cast<double (*)[kSK][TM + 1]>(score_smem + 2 * kSK * (TM + 1));
     const int bh = blockIdx.z;
-    const int i0 = blockIdx.y * kST, j0 = blockIdx.x * kST;
+    const int i0 = blockIdx.y * TM, j0 = blockIdx.x * TM;
     const double* Q = qbar + (size_t)bh * nb * d;
     const double* K = kbar + (size_t)bh * nb * d;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    double acc[4][4] = {};
-    for (int k0 = 0; k0 < d; k0 += kSK) {
-        for (int e = threadIdx.x; e < kST * kSK; e += 256) {
-            const int r = e / kSK, kk = e % kSK;
-            As[kk][r] = (i0 + r < nb) ? Q[(size_t)(i0 + r) * d + k0 + kk] : 0.0;
-            Bs[kk][r] = (j0 + r < nb) ? K[(size_t)(j0 + r) * d + k0 + kk] : 0.0;
+    double acc[R][R];
+#pragma unroll
+    for (int u = 0; u < R; ++u)
+#pragma unroll
+        for (int v = 0; v < R; ++v) acc[u][v] = 0.0;
+    // slice loads: element e = threadIdx.x + 256*l -> (row e / 16, column e % 16); 16 threads read one
+    // row's 128 contiguous bytes
+    double pa[L], pb[L];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int l = 0; l < L; ++l) {
+            const int e = threadIdx.x + 256 * l, rr = e / kSK, kk = e % kSK;
+            pa[l] = (i0 + rr < nb) ? Q[(size_t)(i0 + rr) * d + k0 + kk] : 0.0;
+            pb[l] = (j0 + rr < nb) ? K[(size_t)(j0 + rr) * d + k0 + kk] : 0.0;
         }
-        __syncthreads();
+    };
+    auto stash = [&](int buf) {
+#pragma unroll
+        for (int l = 0; l < L; ++l) {
+            const int e = threadIdx.x + 256 * l, rr = e / kSK, kk = e % kSK;
+            As[buf][kk][rr] = pa[l];
+            Bs[buf][kk][rr] = pb[l];
+        }
+    };
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < d; k0 += kSK) {
+        const bool more = k0 + kSK < d;
+        if (more) fetch(k0 + kSK);                    // in flight while this slice is multiplied
 #pragma unroll
         for (int kk = 0; kk < kSK; ++kk) {
-            double a[4], bv[4];
+            double av[R], bv[R];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) { a[u] = As[kk][ty + 16 * u]; bv[u] = Bs[kk][tx + 16 * u]; }
+            for (int u = 0; u < R; ++u) { av[u] = As[buf][kk][ty + 16 * u]; bv[u] = Bs[buf][kk][tx + 16 * u]; }
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < R; ++u)
 #pragma unroll
-                for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], bv[v], acc[u][v]);
+                for (int v = 0; v < R; ++v) acc[u][v] = fma(av[u], bv[v], acc[u][v]);
         }
+        if (more) stash(buf ^ 1);                     // the other buffer was last read one slice ago
         __syncthreads();
+        buf ^= 1;
     }
     double* out = S + (size_t)bh * nb * nb;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < R; ++u) {
         const int i = i0 + ty + 16 * u;
         if (i >= nb) continue;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
+        for (int v = 0; v < R; ++v) {
             const int j = j0 + tx + 16 * v;
             if (j < nb) out[(size_t)i * nb + j] = acc[u][v] * scale;
         }
@@ -153,100 +184,260 @@ k_scores(const double* __restrict__ qbar, const double* __restrict__ kbar, doubl
 }
 
 // ---------------------------------------------------------------------------
-// Row routing: one CTA per row.  The row's scores are sorted in shared memory
-// by (s desc, j asc) -- softmax is monotone, so this is the order of P -- with
-// a bitonic network over the next power of two; then P_(n), the inclusive
-// cumulative mass, and the smallest n with C_n >= p.
+// Row routing, one warp per row (nb <= 1024).  Each lane holds E = nbp/32
+// consecutive elements of the padded row as one 64-bit key that sorts in
+// ascending order exactly as (s descending, j ascending): the order-preserving
+// image of s, complemented, with its 10 lowest bits replaced by j.  (Dropping
+// those bits only merges scores equal to ~1e-13 relative, far inside the 1e-6
+// tie tolerance, and then orders them by ascending j as the exact rule does.)
+// A bitonic network sorts the keys: exchanges between registers for strides
+// below E, between lanes (shuffles) above.  P, the inclusive cumulative mass
+// and the Top-p cut follow in fp64.
 // ---------------------------------------------------------------------------
-constexpr int kRouteThreads = 256;
-
-__device__ __forceinline__ bool before(double sa, int ja, double sb, int jb) {
-    return sa > sb || (sa == sb && ja < jb);
+constexpr unsigned long long kJMask = 0x1FFFull;          // 13-bit block index field (nb <= 8192)
+constexpr unsigned long long kPadKey = ~0ull & ~kJMask;    // sorts after every real score
+__device__ __forceinline__ unsigned long long desc_key(double s, int j) {
+    unsigned long long u = (unsigned long long)__double_as_longlong(s);
+    u = (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);   // ascending with s
+    return (~u & ~kJMask) | (unsigned long long)j;
+}
+__device__ __forceinline__ double key_score(unsigned long long key) {
+    unsigned long long u = ~(key | kJMask);                          // low bits of s are gone
+    u = (u & 0x8000000000000000ull) ? (u & 0x7FFFFFFFFFFFFFFFull) : ~u;
+    return __longlong_as_double((long long)u);
 }
 
-template <typename Op>
-__device__ double block_reduce(double v, double* red, Op op) {
-    for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-    __syncthreads();
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    v = red[0];
-    for (int u = 1; u < (int)(blockDim.x / 32); ++u) v = op(v, red[u]);
-    return v;
-}
-
-__global__ void __launch_bounds__(kRouteThreads)
-k_route_rows(const double* __restrict__ S, int nb, int nbp, double p, int k_floor,
+template <int E>
+__global__ void __launch_bounds__(128, 1)
+k_route_warp(const double* __restrict__ S, int64_t rows, int nb, double p, int k_floor,
              uint16_t* __restrict__ sorted, int32_t* __restrict__ counts) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    double* key = reinterpret_cast<double*>(smem_raw);            // [nbp]
-    int* idx = reinterpret_cast<int*>(key + nbp);                 // [nbp]
-    __shared__ double red[kRouteThreads / 32];
-    __shared__ double wsum[kRouteThreads / 32];
-    __shared__ int s_np;
-    const size_t r = blockIdx.x;
+    constexpr int NBP = 32 * E;
+    constexpr int LOGN = E == 1 ? 5 : E == 2 ? 6 : E == 4 ? 7 : E == 8 ? 8 : E == 16 ? 9 : 10;
+    static_assert((1 << LOGN) == NBP, "E must be a power of two <= 32");
+    const int lane = threadIdx.x % 32;
+    const int64_t r = (int64_t)blockIdx.x * 4 + threadIdx.x / 32;
+    if (r >= rows) return;
     const double* row = S + r * nb;
-    const int tid = threadIdx.x;
-
+    unsigned long long key[E];
     double mx = -INFINITY;
-    for (int j = tid; j < nbp; j += blockDim.x) {
-        const double s = j < nb ? row[j] : -INFINITY;
-        key[j] = s;
-        idx[j] = j;
-        mx = fmax(mx, s);
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int e = lane * E + k;
+        if (e < nb) {
+            const double sv = row[e];
+            mx = fmax(mx, sv);
+            key[k] = desc_key(sv, e);
+        } else {
+            key[k] = kPadKey | (unsigned long long)(e & kJMask);               // after every score
+        }
     }
-    mx = block_reduce(mx, red, [](double a, double b) { return fmax(a, b); });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     double z = 0.0;
-    for (int j = tid; j < nb; j += blockDim.x) z += exp(key[j] - mx);
-    z = block_reduce(z, red, [](double a, double b) { return a + b; });
+#pragma unroll
+    for (int k = 0; k < E; ++k) z += (lane * E + k < nb) ? exp(key_score(key[k]) - mx) : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 
-    // bitonic sort, "before" order first
-    for (int size = 2; size <= nbp; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            __syncthreads();
-            for (int t = tid; t < nbp / 2; t += blockDim.x) {
-                const int a = 2 * t - (t & (stride - 1));
-                const int b = a + stride;
-                const bool up = (a & size) == 0;       // this half sorts in "before" order
-                const double ka = key[a], kb = key[b];
-                const int ia = idx[a], ib = idx[b];
-                const bool swap = up ? before(kb, ib, ka, ia) : before(ka, ia, kb, ib);
-                if (swap) { key[a] = kb; key[b] = ka; idx[a] = ib; idx[b] = ia; }
+    // bitonic sort, ascending keys; every loop bound is a compile-time constant
+#pragma unroll
+    for (int ls = 1; ls <= LOGN; ++ls) {
+#pragma unroll
+        for (int lt = ls - 1; lt >= 0; --lt) {
+            const int size = 1 << ls, stride = 1 << lt;
+            if (stride < E) {
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    if ((k & stride) == 0) {
+                        const int kp = k | stride;
+                        const bool up = ((lane * E + k) & size) == 0;
+                        const unsigned long long a = key[k], b = key[kp];
+                        const bool sw = up ? (b < a) : (a < b);
+                        key[k] = sw ? b : a;
+                        key[kp] = sw ? a : b;
+                    }
+                }
+            } else {
+                const int lmask = stride / E;
+                const bool lower = (lane & lmask) == 0;
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    const bool up = ((lane * E + k) & size) == 0;
+                    const unsigned long long mine = key[k];
+                    const unsigned long long other = __shfl_xor_sync(0xffffffffu, mine, lmask);
+                    key[k] = ((other < mine) == (lower == up)) ? other : mine;
+                }
             }
         }
     }
-    __syncthreads();
-
-    // P in sorted order, inclusive scan: each thread owns a contiguous run
-    const int per = (nbp + blockDim.x - 1) / blockDim.x;
-    const int lo = tid * per, hi = min(nb, lo + per);
+    // P in sorted order, inclusive cumulative mass, first n with C_n >= p
+    double c[E];
     double run = 0.0;
-    for (int n = lo; n < hi; ++n) { const double pn = exp(key[n] - mx) / z; run += pn; key[n] = run; }
-    // exclusive scan of per-thread totals
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int e = lane * E + k;
+        run += e < nb ? exp(key_score(key[k]) - mx) / z : 0.0;
+        c[k] = run;
+    }
+    double excl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, excl, o);
+        if (lane >= o) excl += y;
+    }
+    excl -= run;
+    int first = nb;
+#pragma unroll
+    for (int k = E - 1; k >= 0; --k) {
+        const int e = lane * E + k;
+        if (e < nb && c[k] + excl >= p) first = e + 1;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    const int n_p = p >= 1.0 ? nb : first;
+    const int n_i = min(nb, max(k_floor, n_p));
+    uint16_t* dst = sorted + r * nb;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int e = lane * E + k;
+        if (e < n_i) dst[e] = (uint16_t)(key[k] & kJMask);
+    }
+    if (lane == 0) counts[r] = n_i;
+}
+
+// ---------------------------------------------------------------------------
+// Row routing for long rows (nbp >= 512): one 256-thread CTA per row, E =
+// nbp/256 keys per thread (same keys as above).  Bitonic exchanges run inside
+// a thread's registers for strides below E, by warp shuffle for strides below
+// 32E, and through shared memory above (two barriers per such stage).
+// ---------------------------------------------------------------------------
+constexpr int kCtaSortThreads = 256;
+
+template <int E>
+__global__ void __launch_bounds__(kCtaSortThreads)
+k_route_cta(const double* __restrict__ S, int nb, double p, int k_floor,
+            uint16_t* __restrict__ sorted, int32_t* __restrict__ counts) {
+    constexpr int NBP = kCtaSortThreads * E;
+    constexpr int LOGN = E == 2 ? 9 : E == 4 ? 10 : E == 8 ? 11 : E == 16 ? 12 : 13;
+    static_assert((1 << LOGN) == NBP, "E must be 2, 4, 8, 16 or 32");
+    extern __shared__ unsigned long long xk[];              // [NBP] cross-warp exchange
+    __shared__ double red[kCtaSortThreads / 32];
+    __shared__ int s_first;
+    const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
+    const size_t r = blockIdx.x;
+    const double* row = S + r * nb;
+    unsigned long long key[E];
+    double mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int e = tid * E + k;
+        if (e < nb) {
+            const double sv = row[e];
+            mx = fmax(mx, sv);
+            key[k] = desc_key(sv, e);
+        } else {
+            key[k] = kPadKey | (unsigned long long)(e & kJMask);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[wid] = mx;
+    if (tid == 0) s_first = nb;
+    __syncthreads();
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < kCtaSortThreads / 32; ++w) mx = fmax(mx, red[w]);
+    double z = 0.0;
+#pragma unroll
+    for (int k = 0; k < E; ++k) z += (tid * E + k < nb) ? exp(key_score(key[k]) - mx) : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    __syncthreads();                                         // everyone has read red[] (max)
+    if (lane == 0) red[wid] = z;
+    __syncthreads();
+    z = 0.0;
+#pragma unroll
+    for (int w = 0; w < kCtaSortThreads / 32; ++w) z += red[w];
+
+#pragma unroll
+    for (int ls = 1; ls <= LOGN; ++ls) {
+#pragma unroll
+        for (int lt = ls - 1; lt >= 0; --lt) {
+            const int size = 1 << ls, stride = 1 << lt;
+            if (stride < E) {
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    if ((k & stride) == 0) {
+                        const int kp = k | stride;
+                        const bool up = ((tid * E + k) & size) == 0;
+                        const unsigned long long a = key[k], b = key[kp];
+                        const bool sw = up ? (b < a) : (a < b);
+                        key[k] = sw ? b : a;
+                        key[kp] = sw ? a : b;
+                    }
+                }
+            } else if (stride < 32 * E) {
+                const int lmask = stride / E;
+                const bool lower = (lane & lmask) == 0;
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    const bool up = ((tid * E + k) & size) == 0;
+                    const unsigned long long mine = key[k];
+                    const unsigned long long other = __shfl_xor_sync(0xffffffffu, mine, lmask);
+                    key[k] = ((other < mine) == (lower == up)) ? other : mine;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < E; ++k) xk[tid * E + k] = key[k];
+                __syncthreads();
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    const int e = tid * E + k;
+                    const bool up = (e & size) == 0, lower = (e & stride) == 0;
+                    const unsigned long long mine = key[k], other = xk[e ^ stride];
+                    key[k] = ((other < mine) == (lower == up)) ? other : mine;
+                }
+                __syncthreads();
+            }
+        }
+    }
+    // P in sorted order, inclusive cumulative mass, first n with C_n >= p
+    double c[E];
+    double run = 0.0;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int e = tid * E + k;
+        run += e < nb ? exp(key_score(key[k]) - mx) / z : 0.0;
+        c[k] = run;
+    }
     double incl = run;
-    const int lane = tid % 32, wid = tid / 32;
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const double y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
     }
-    if (lane == 31) wsum[wid] = incl;
-    if (tid == 0) s_np = nb;
+    if (lane == 31) red[wid] = incl;                        // red[] free: z was read before the sort
     __syncthreads();
-    double off = incl - run;
-    for (int w = 0; w < wid; ++w) off += wsum[w];
+    double excl = incl - run;
+    for (int w = 0; w < wid; ++w) excl += red[w];
     int first = nb;
-    for (int n = lo; n < hi; ++n) {
-        const double c = key[n] + off;
-        if (c >= p) { first = n + 1; break; }
+#pragma unroll
+    for (int k = E - 1; k >= 0; --k) {
+        const int e = tid * E + k;
+        if (e < nb && c[k] + excl >= p) first = e + 1;
     }
-    if (first < nb) atomicMin(&s_np, first);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    if (lane == 0 && first < nb) atomicMin(&s_first, first);
     __syncthreads();
-    int n_p = s_np;
-    if (p >= 1.0) n_p = nb;
+    const int n_p = p >= 1.0 ? nb : s_first;
     const int n_i = min(nb, max(k_floor, n_p));
     uint16_t* dst = sorted + r * nb;
-    for (int n = tid; n < n_i; n += blockDim.x) dst[n] = (uint16_t)idx[n];
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int e = tid * E + k;
+        if (e < n_i) dst[e] = (uint16_t)(key[k] & kJMask);
+    }
     if (tid == 0) counts[r] = n_i;
 }
 
@@ -258,30 +449,35 @@ constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads)
 k_csr_scan(const int32_t* __restrict__ counts, int64_t rows, int nb, int32_t* __restrict__ row_ptr,
            float* __restrict__ L_h, int64_t* __restrict__ nnz, int64_t col_cap, int32_t* err) {
+    // chunks of kScanThreads rows: coalesced loads, block-wide scan, running offset
     __shared__ long long wsum[kScanThreads / 32];
-    const int tid = threadIdx.x;
-    const int64_t per = (rows + kScanThreads - 1) / kScanThreads;
-    const int64_t lo = tid * per, hi = min(rows, lo + per);
-    long long run = 0;
-    for (int64_t r = lo; r < hi; ++r) run += counts[r];
-    long long incl = run;
-    const int lane = tid % 32, wid = tid / 32;
-    for (int o = 1; o < 32; o <<= 1) {
-        const long long y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) wsum[wid] = incl;
+    __shared__ long long s_carry;
+    const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
+    if (tid == 0) s_carry = 0;
     __syncthreads();
-    long long off = incl - run;
-    for (int w = 0; w < wid; ++w) off += wsum[w];
-    for (int64_t r = lo; r < hi; ++r) {
-        row_ptr[r] = (int32_t)off;
-        off += counts[r];
+    for (int64_t base = 0; base < rows; base += kScanThreads) {
+        const int64_t r = base + tid;
+        const long long v = r < rows ? counts[r] : 0;
+        long long incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[wid] = incl;
+        __syncthreads();
+        long long off = s_carry;
+        for (int w = 0; w < wid; ++w) off += wsum[w];
+        if (r < rows) row_ptr[r] = (int32_t)(off + incl - v);
+        __syncthreads();                                   // all reads of wsum / s_carry done
+        if (tid == kScanThreads - 1) s_carry = off + incl;
+        __syncthreads();
     }
-    if (tid == kScanThreads - 1) {
-        row_ptr[rows] = (int32_t)off;
-        *nnz = off;
-        if (off > col_cap) record_error(err, BSA_ECAPACITY, 0);
+    const long long total = s_carry;
+    if (tid == 0) {
+        row_ptr[rows] = (int32_t)total;
+        *nnz = total;
+        if (total > col_cap) record_error(err, BSA_ECAPACITY, 0);
     }
     __syncthreads();
     // L_h: integer sum over a head's rows, then one fp32 divide (Eq. 1)
@@ -308,22 +504,37 @@ cudaError_t launch_pool(const bsa_plan& p, const void* q, const void* k, int dty
                         double* qbar, double* kbar, cudaStream_t s) {
     const int V = dtype == BSA_BF16 ? 8 : 4;
     const int chunks = (p.H * p.d) / V;
-    dim3 grid((unsigned)p.nb, (unsigned)((chunks + kPoolThreads - 1) / kPoolThreads), (unsigned)(2 * p.B));
+    const int threads = chunks >= kPoolThreads ? kPoolThreads : (chunks + 31) / 32 * 32;
+    dim3 grid((unsigned)p.nb, (unsigned)((chunks + threads - 1) / threads), (unsigned)(2 * p.B));
     if (dtype == BSA_BF16)
-        k_pool<__nv_bfloat16><<<grid, kPoolThreads, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                           p.d_perm, qbar, kbar, (int)p.N, p.H, p.d, p.block, (int)p.nb);
+        k_pool<__nv_bfloat16><<<grid, threads, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                       p.d_perm, qbar, kbar, (int)p.N, p.H, p.d, p.block, (int)p.nb);
     else
-        k_pool<float><<<grid, kPoolThreads, 0, s>>>((const float*)q, (const float*)k, p.d_perm, qbar, kbar,
-                                                   (int)p.N, p.H, p.d, p.block, (int)p.nb);
+        k_pool<float><<<grid, threads, 0, s>>>((const float*)q, (const float*)k, p.d_perm, qbar, kbar,
+                                               (int)p.N, p.H, p.d, p.block, (int)p.nb);
+    return cudaGetLastError();
+}
+
+template <int TM>
+cudaError_t launch_scores_tm(const bsa_plan& p, const double* qbar, const double* kbar, double* scores,
+                             cudaStream_t s, double scale) {
+    const int smem = 4 * kSK * (TM + 1) * (int)sizeof(double);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_scores<TM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int t = (int)((p.nb + TM - 1) / TM);
+    dim3 grid(t, t, (unsigned)(p.B * p.H));
+    k_scores<TM><<<grid, 256, smem, s>>>(qbar, kbar, scores, (int)p.nb, p.d, scale);
     return cudaGetLastError();
 }
 
 cudaError_t launch_scores(const bsa_plan& p, const double* qbar, const double* kbar, double* scores,
                           cudaStream_t s) {
-    const int t = (int)((p.nb + kST - 1) / kST);
-    dim3 grid(t, t, (unsigned)(p.B * p.H));
-    k_scores<<<grid, 256, 0, s>>>(qbar, kbar, scores, (int)p.nb, p.d, 1.0 / sqrt((double)p.d));
-    return cudaGetLastError();
+    const double scale = 1.0 / sqrt((double)p.d);
+    const int64_t t128 = (p.nb + 127) / 128;
+    if (t128 * t128 * p.B * p.H >= 2 * p.num_sms) return launch_scores_tm<128>(p, qbar, kbar, scores, s, scale);
+    return launch_scores_tm<64>(p, qbar, kbar, scores, s, scale);
 }
 
 cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pval, int k_floor,
@@ -331,13 +542,34 @@ cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pv
     int nbp = 1;
     while (nbp < p.nb) nbp <<= 1;
     nbp = nbp < 2 ? 2 : nbp;
-    const size_t smem = (size_t)nbp * (sizeof(double) + sizeof(int));
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_route_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
+    const int nb = (int)p.nb;
+    if (nbp <= 256) {
+        const unsigned grid = (unsigned)((p.rows + 3) / 4);
+        switch (nbp <= 32 ? 1 : nbp / 32) {
+            case 1: k_route_warp<1><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
+            case 2: k_route_warp<2><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
+            case 4: k_route_warp<4><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
+            default: k_route_warp<8><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
+        }
+        return cudaGetLastError();
     }
-    k_route_rows<<<(unsigned)p.rows, kRouteThreads, smem, s>>>(scores, (int)p.nb, nbp, pval, k_floor, sorted, counts);
-    return cudaGetLastError();
+    const int E = nbp / kCtaSortThreads;
+    const size_t smem = (size_t)nbp * sizeof(unsigned long long);
+    auto run = [&](auto kern) -> cudaError_t {
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        kern<<<(unsigned)p.rows, kCtaSortThreads, smem, s>>>(scores, nb, pval, k_floor, sorted, counts);
+        return cudaGetLastError();
+    };
+    switch (E) {
+        case 2: return run(k_route_cta<2>);
+        case 4: return run(k_route_cta<4>);
+        case 8: return run(k_route_cta<8>);
+        case 16: return run(k_route_cta<16>);
+        default: return run(k_route_cta<32>);
+    }
 }
 
 cudaError_t launch_csr(const bsa_plan& p, const int32_t* counts, const uint16_t* sorted, int32_t* row_ptr,

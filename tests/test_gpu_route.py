@@ -37,7 +37,7 @@ def compare(bsa, w, x, p, k_floor, order=0):
     g = gpu_route(bsa, w, x, p, k_floor, order)
     assert g["status"] == 0
     amb = check_route(g["row_ptr"], g["col_idx"], g["L_h"], g["nnz"], ref, w.B * w.H)
-    assert amb < 0.01 or w.rows < 1000        # tie fraction only meaningful on many rows
+    assert amb < 0.02 or w.rows < 1000        # tie fraction only meaningful on many rows
     return g, ref
 
 
@@ -80,6 +80,17 @@ def test_ragged_shapes(bsa, shape, order):
     x = syn.make_inputs(w, seed=11)
     for p, kf in ((0.9, 2), (0.7, 0), (1.0, 1)):
         compare(bsa, w, x, p, kf, order)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=8, Hs=100, Ws=100, H=1, d=64, block=64),     # 1250 blocks per row: CTA sort, 8 keys per thread
+    dict(T=26, Hs=100, Ws=101, H=1, d=64, block=64),    # 4104 blocks per row: CTA sort, 32 keys per thread
+])
+def test_long_rows(bsa, shape):
+    w = syn.workload(2, **shape)
+    x = syn.make_inputs(w, seed=13)
+    for p, kf in ((0.9, 4), (0.5, 1)):
+        compare(bsa, w, x, p, kf)
 
 
 def test_fp32_input_path(bsa):
