@@ -63,6 +63,18 @@ def attention_flops(row_ptr, col_idx, w):
     return 4.0 * w.d * float(np.sum(m[rows % w.nb] * m[cols]))
 
 
+def reduce_over_ranks(times_ms, work, world, device):
+    """Whole-job view of a replicated run: the max over ranks of each timing and
+    the sum over ranks of the work.  Every rank takes the same two collectives."""
+    import torch
+    stats = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    total = torch.tensor([float(work)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(total, op=torch.distributed.ReduceOp.SUM)
+    return [float(x) for x in stats.tolist()], float(total[0])
+
+
 def route_bytes(w, nnz, in_bytes):
     return 2 * in_bytes + (w.rows + 1) * 4 + nnz * 4 + w.B * w.H * 4 + 8
 
@@ -207,13 +219,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    stats = torch.tensor([total_ms, e2e_ms, max(attn_ms), max(route_ms)], dtype=torch.float64, device=dev)
-    flops_all = torch.tensor([flops], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
-        torch.distributed.all_reduce(flops_all, op=torch.distributed.ReduceOp.SUM)
-    total_ms_max, e2e_ms_max = float(stats[0]), float(stats[1])
-    flops_sum = float(flops_all[0])
+    (total_ms_max, e2e_ms_max, _, _), flops_sum = reduce_over_ranks(
+        [total_ms, e2e_ms, max(attn_ms), max(route_ms)], flops, world, dev)
     if rank != 0:
         return None
 

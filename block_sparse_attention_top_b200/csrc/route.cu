@@ -449,16 +449,20 @@ constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads)
 k_csr_scan(const int32_t* __restrict__ counts, int64_t rows, int nb, int32_t* __restrict__ row_ptr,
            float* __restrict__ L_h, int64_t* __restrict__ nnz, int64_t col_cap, int32_t* err) {
-    // chunks of kScanThreads rows: coalesced loads, block-wide scan, running offset
+    // chunks of 4*kScanThreads rows (4 consecutive rows per thread): block-wide
+    // scan of the per-thread sums, running offset carried between chunks
     __shared__ long long wsum[kScanThreads / 32];
     __shared__ long long s_carry;
     const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
     if (tid == 0) s_carry = 0;
     __syncthreads();
-    for (int64_t base = 0; base < rows; base += kScanThreads) {
-        const int64_t r = base + tid;
-        const long long v = r < rows ? counts[r] : 0;
-        long long incl = v;
+    for (int64_t base = 0; base < rows; base += 4 * kScanThreads) {
+        const int64_t r0 = base + 4 * (int64_t)tid;
+        long long v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = r0 + u < rows ? counts[r0 + u] : 0;
+        const long long mine = v[0] + v[1] + v[2] + v[3];
+        long long incl = mine;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const long long y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -466,11 +470,15 @@ k_csr_scan(const int32_t* __restrict__ counts, int64_t rows, int nb, int32_t* __
         }
         if (lane == 31) wsum[wid] = incl;
         __syncthreads();
-        long long off = s_carry;
+        long long off = s_carry + incl - mine;
         for (int w = 0; w < wid; ++w) off += wsum[w];
-        if (r < rows) row_ptr[r] = (int32_t)(off + incl - v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (r0 + u < rows) row_ptr[r0 + u] = (int32_t)off;
+            off += v[u];
+        }
         __syncthreads();                                   // all reads of wsum / s_carry done
-        if (tid == kScanThreads - 1) s_carry = off + incl;
+        if (tid == kScanThreads - 1) s_carry = off;
         __syncthreads();
     }
     const long long total = s_carry;
