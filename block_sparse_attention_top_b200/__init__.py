@@ -30,7 +30,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 BSA_OK, BSA_EINVAL, BSA_EUNSUPPORTED, BSA_ECAPACITY, BSA_EWORKSPACE, BSA_ECUDA, BSA_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 BSA_ORDER_HILBERT2D_FRAME, BSA_ORDER_IDENTITY = 0, 1
 BSA_BF16, BSA_F32 = 0, 1
-BSA_OP_ROUTE, BSA_OP_ATTN = 0, 1
+BSA_OP_ROUTE, BSA_OP_ATTN, BSA_OP_MASK, BSA_OP_AUGMENT = 0, 1, 2, 3
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -46,6 +46,10 @@ _SIGS = {
     "bsa_route": (_I, [_P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
     "bsa_route_static": (_I, [_P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _I64, _P, _P, _P]),
     "bsa_route_intermediates": (_I, [_P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P)]),
+    "bsa_mask_window_anchor": (_I, [_P, _I, _I, _I, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "bsa_route_order": (_I, [_P, _P, ctypes.POINTER(_P)]),
+    "bsa_augment": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
+    "bsa_sasa_budget": (_I, [_I, _P, ctypes.c_float, ctypes.c_float, ctypes.c_float, _P, _P, _P, _P, _P]),
     "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_run": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
@@ -138,6 +142,43 @@ def bsa_route_static(plan, q, k, dtype, p, k_floor, row_ptr, col_idx, col_cap, L
     (for callers that cannot allocate when they route)."""
     return _lib.bsa_route_static(plan.handle, _ptr(q), _ptr(k), dtype, float(p), int(k_floor), _ptr(row_ptr),
                                  _ptr(col_idx), int(col_cap), _ptr(L_h), _ptr(nnz), _stream(stream))
+
+
+def bsa_mask_window_anchor(plan, radius_frames, n_anchor, step, row_ptr, col_idx, col_cap, nnz, workspace,
+                           stream=None):
+    return _lib.bsa_mask_window_anchor(plan.handle, int(radius_frames), int(n_anchor), int(step), _ptr(row_ptr),
+                                       _ptr(col_idx), int(col_cap), _ptr(nnz), _ptr(workspace),
+                                       workspace.numel() if workspace is not None else 0, _stream(stream))
+
+
+def bsa_route_order(plan, workspace):
+    """Device address of the full importance order (uint16 [rows, nb]) in a route workspace."""
+    out = _P()
+    _check(_lib.bsa_route_order(plan.handle, _ptr(workspace), ctypes.byref(out)), "bsa_route_order")
+    return out.value
+
+
+def bsa_augment(plan, row_ptr, order, extra, row_ptr_out, col_idx_out, col_cap, L_h_out, nnz_out, workspace,
+                stream=None):
+    return _lib.bsa_augment(plan.handle, _ptr(row_ptr), _ptr(order), _ptr(extra), _ptr(row_ptr_out),
+                            _ptr(col_idx_out), int(col_cap), _ptr(L_h_out), _ptr(nnz_out), _ptr(workspace),
+                            workspace.numel() if workspace is not None else 0, _stream(stream))
+
+
+def bsa_sasa_budget(L_r, n1=0.8, n2=0.07, S=0.0, heads_per_rank=None):
+    """Host-only SASA budget (Eqs. 7-10).  Returns (B_r, L_aug, A, extra_per_head or None)."""
+    R = len(L_r)
+    L = torch.tensor(list(L_r), dtype=torch.float32)
+    B = torch.empty(R, dtype=torch.float32)
+    La = torch.empty(R, dtype=torch.float32)
+    A = torch.empty(1, dtype=torch.float32)
+    hp = ex = None
+    if heads_per_rank is not None:
+        hp = torch.tensor(list(heads_per_rank), dtype=torch.int32)
+        ex = torch.empty(int(hp.sum()), dtype=torch.int32)
+    _check(_lib.bsa_sasa_budget(R, L.data_ptr(), float(n1), float(n2), float(S), B.data_ptr(), La.data_ptr(),
+                                A.data_ptr(), _ptr(hp), _ptr(ex)), "bsa_sasa_budget")
+    return B, La, float(A[0]), ex
 
 
 def bsa_route_intermediates(plan, workspace):

@@ -165,6 +165,7 @@ size_t bsa_workspace_size(const bsa_plan* p, int op) {
     if (!p) return 0;
     if (op == BSA_OP_ROUTE) return route_ws_layout(*p).total;
     if (op == BSA_OP_ATTN) return attn_ws_layout(*p).total;
+    if (op == BSA_OP_MASK || op == BSA_OP_AUGMENT) return mask_ws_bytes(*p);
     return 0;
 }
 
@@ -199,6 +200,64 @@ int bsa_route(const bsa_plan* p, const void* q, const void* k, int dtype, float 
     BSA_LAUNCH(launch_scores(*p, qbar, kbar, scores, s));
     BSA_LAUNCH(launch_route_rows(*p, scores, (double)pval, k_floor, sorted, counts, s));
     BSA_LAUNCH(launch_csr(*p, counts, sorted, row_ptr, col_idx, col_cap, L_h, nnz, s));
+    return BSA_OK;
+}
+
+int bsa_route_order(const bsa_plan* p, void* ws, const uint16_t** order) {
+    if (!p || !ws || !order) return BSA_EINVAL;
+    *order = (const uint16_t*)((char*)ws + route_ws_layout(*p).sorted);
+    return BSA_OK;
+}
+
+int bsa_augment(const bsa_plan* p, const int32_t* row_ptr, const uint16_t* order, const int32_t* extra,
+                int32_t* row_ptr_out, int32_t* col_idx_out, int64_t col_cap, float* L_h_out, int64_t* nnz_out,
+                void* ws, size_t ws_bytes, void* stream) {
+    if (!p || !row_ptr || !order || !extra || !row_ptr_out || !L_h_out || !nnz_out) return BSA_EINVAL;
+    if (col_cap < 0 || (col_cap > 0 && !col_idx_out)) return BSA_EINVAL;
+    if (misaligned(row_ptr, 4) || misaligned(order, 2) || misaligned(extra, 4) || misaligned(row_ptr_out, 4) ||
+        (col_idx_out && misaligned(col_idx_out, 4)) || misaligned(L_h_out, 4) || misaligned(nnz_out, 8))
+        return BSA_EINVAL;
+    if (int rc = check_ws(ws, ws_bytes, mask_ws_bytes(*p))) return rc;
+    BSA_LAUNCH(launch_augment(*p, row_ptr, order, extra, (int32_t*)ws, row_ptr_out, col_idx_out, col_cap, L_h_out,
+                              nnz_out, (cudaStream_t)stream));
+    return BSA_OK;
+}
+
+int bsa_sasa_budget(int R, const float* L_r, float n1, float n2, float S, float* B_r, float* L_aug, float* A,
+                    const int32_t* heads_per_rank, int32_t* extra_per_head) {
+    if (R < 1 || !L_r || !B_r) return BSA_EINVAL;
+    if (heads_per_rank && !extra_per_head) return BSA_EINVAL;
+    double lmax = L_r[0];
+    for (int r = 1; r < R; ++r) lmax = std::max(lmax, (double)L_r[r]);
+    double amax = -1e300;
+    int64_t h = 0;
+    for (int r = 0; r < R; ++r) {
+        const double dl = lmax - (double)L_r[r];
+        const double b = dl > (double)n2 * lmax ? (double)n1 * dl : 0.0;
+        B_r[r] = (float)b;
+        const double la = (double)L_r[r] + b;
+        if (L_aug) L_aug[r] = (float)la;
+        amax = std::max(amax, la);
+        if (heads_per_rank) {
+            if (heads_per_rank[r] < 1) return BSA_EINVAL;
+            const int32_t e = (int32_t)std::floor(b / heads_per_rank[r]);
+            for (int32_t t = 0; t < heads_per_rank[r]; ++t) extra_per_head[h++] = e;
+        }
+    }
+    if (A) *A = (float)(std::max(0.0, amax - lmax) + (double)S);
+    return BSA_OK;
+}
+
+int bsa_mask_window_anchor(const bsa_plan* p, int radius_frames, int n_anchor, int step, int32_t* row_ptr,
+                           int32_t* col_idx, int64_t col_cap, int64_t* nnz, void* ws, size_t ws_bytes,
+                           void* stream) {
+    if (!p || !row_ptr || !nnz || radius_frames < 0 || n_anchor < 0 || n_anchor > kMaxMaskAnchors || step < 0)
+        return BSA_EINVAL;
+    if (col_cap < 0 || (col_cap > 0 && !col_idx)) return BSA_EINVAL;
+    if (misaligned(row_ptr, 4) || (col_idx && misaligned(col_idx, 4)) || misaligned(nnz, 8)) return BSA_EINVAL;
+    if (int rc = check_ws(ws, ws_bytes, mask_ws_bytes(*p))) return rc;
+    BSA_LAUNCH(launch_mask_window_anchor(*p, radius_frames, n_anchor, step, (int32_t*)ws, row_ptr, col_idx, col_cap,
+                                         nnz, (cudaStream_t)stream));
     return BSA_OK;
 }
 

@@ -30,6 +30,9 @@ struct RouteWs {
 RouteWs route_ws_layout(const bsa_plan& p);
 
 // ---- attention workspace layout ----
+// ---- mask workspace: per-row counts ----
+inline size_t mask_ws_bytes(const bsa_plan& p) { return align_up((size_t)p.rows * sizeof(int32_t)); }
+
 struct AttnWs {
     size_t qp, kp, vp, work, hist, bins, counter, total;
 };
@@ -50,6 +53,18 @@ cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pv
 cudaError_t launch_csr(const bsa_plan& p, const int32_t* counts, const uint16_t* sorted,
                        int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, float* L_h,
                        int64_t* nnz, cudaStream_t s);
+
+// Exclusive scan of per-row counts -> row_ptr, nnz (and L_h unless null);
+// BSA_ECAPACITY in the error word when nnz > col_cap.
+cudaError_t launch_scan_counts(const bsa_plan& p, const int32_t* counts, int32_t* row_ptr, float* L_h,
+                               int64_t* nnz, int64_t col_cap, cudaStream_t s);
+cudaError_t launch_mask_window_anchor(const bsa_plan& p, int radius, int n_anchor, int step, int32_t* counts,
+                                      int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, int64_t* nnz,
+                                      cudaStream_t s);
+constexpr int kMaxMaskAnchors = 64;
+cudaError_t launch_augment(const bsa_plan& p, const int32_t* row_ptr, const uint16_t* order, const int32_t* extra,
+                           int32_t* counts, int32_t* row_ptr_out, int32_t* col_idx_out, int64_t col_cap,
+                           float* L_h_out, int64_t* nnz_out, cudaStream_t s);
 
 cudaError_t launch_worklist(const bsa_plan& p, const int32_t* row_ptr, int32_t* hist,
                             int32_t* bins, int32_t* work, cudaStream_t s);

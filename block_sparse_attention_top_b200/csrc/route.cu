@@ -300,7 +300,7 @@ k_route_warp(const double* __restrict__ S, int64_t rows, int nb, double p, int k
 #pragma unroll
     for (int k = 0; k < E; ++k) {
         const int e = lane * E + k;
-        if (e < n_i) dst[e] = (uint16_t)(key[k] & kJMask);
+        if (e < nb) dst[e] = (uint16_t)(key[k] & kJMask);     // the full importance order
     }
     if (lane == 0) counts[r] = n_i;
 }
@@ -436,7 +436,7 @@ k_route_cta(const double* __restrict__ S, int nb, double p, int k_floor,
 #pragma unroll
     for (int k = 0; k < E; ++k) {
         const int e = tid * E + k;
-        if (e < n_i) dst[e] = (uint16_t)(key[k] & kJMask);
+        if (e < nb) dst[e] = (uint16_t)(key[k] & kJMask);     // the full importance order
     }
     if (tid == 0) counts[r] = n_i;
 }
@@ -489,6 +489,7 @@ k_csr_scan(const int32_t* __restrict__ counts, int64_t rows, int nb, int32_t* __
     }
     __syncthreads();
     // L_h: integer sum over a head's rows, then one fp32 divide (Eq. 1)
+    if (L_h == nullptr) return;
     const int64_t heads = rows / nb;
     for (int64_t bh = tid; bh < heads; bh += kScanThreads)
         L_h[bh] = (float)(row_ptr[(bh + 1) * nb] - row_ptr[bh * nb]) / (float)nb;
@@ -578,6 +579,12 @@ cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pv
         case 16: return run(k_route_cta<16>);
         default: return run(k_route_cta<32>);
     }
+}
+
+cudaError_t launch_scan_counts(const bsa_plan& p, const int32_t* counts, int32_t* row_ptr, float* L_h,
+                               int64_t* nnz, int64_t col_cap, cudaStream_t s) {
+    k_csr_scan<<<1, kScanThreads, 0, s>>>(counts, p.rows, (int)p.nb, row_ptr, L_h, nnz, col_cap, p.d_err);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_csr(const bsa_plan& p, const int32_t* counts, const uint16_t* sorted, int32_t* row_ptr,

@@ -66,6 +66,8 @@ extern "C" {
 /* ---- workspace queries ---- */
 #define BSA_OP_ROUTE 0
 #define BSA_OP_ATTN  1
+#define BSA_OP_MASK  2
+#define BSA_OP_AUGMENT 3
 
 typedef struct bsa_plan bsa_plan;
 
@@ -96,8 +98,9 @@ int bsa_plan_info(const bsa_plan* plan, int64_t* N, int64_t* nb, int64_t* rows);
  */
 int bsa_token_order(int T, int Hs, int Ws, int order, int32_t* perm);
 
-/* Bytes of device workspace that bsa_route (BSA_OP_ROUTE) or bsa_sparse_attn
- * (BSA_OP_ATTN) needs for this plan; 0 for a NULL plan or unknown op. */
+/* Bytes of device workspace that bsa_route (BSA_OP_ROUTE), bsa_sparse_attn
+ * (BSA_OP_ATTN), bsa_mask_window_anchor (BSA_OP_MASK) or
+ * bsa_augment (BSA_OP_AUGMENT); 0 for a NULL plan or unknown op. */
 size_t bsa_workspace_size(const bsa_plan* plan, int op);
 
 /*
@@ -154,6 +157,61 @@ int bsa_route_static(const bsa_plan* plan, const void* q, const void* k, int dty
 int bsa_route_intermediates(const bsa_plan* plan, void* workspace,
                             const double** qbar, const double** kbar,
                             const double** scores);
+
+/*
+ * Device pointer to the full key-block importance order the last bsa_route
+ * left in `workspace`: uint16 [rows, nb],
+ * row r = every key block of the row in descending block mass (equal mass:
+ * ascending j) -- the review's Stage-1 "key-block importance order" output.
+ * The first n_i entries of a row are its routed columns.  Valid until the next
+ * routing call on the same workspace.  No CUDA call.
+ */
+int bsa_route_order(const bsa_plan* plan, void* workspace, const uint16_t** order);
+
+/*
+ * Slack-aware augmentation, the in-place step of the review's SASA (section 3
+ * "Stage 3" and its algorithm flow): every query block of head bh keeps its
+ * routed blocks and gains the next extra[bh] blocks of its importance order
+ * (clamped at nb); no re-scoring, no re-sorting.  row_ptr: the routed CSR's
+ * row_ptr (its counts are the routed prefixes of `order`); order: from
+ * bsa_route_order; extra: int32 [B*H] on the device (values < 0 act as 0).
+ * Outputs: a new CSR (row_ptr_out [rows+1], col_idx_out [col_cap], columns in
+ * importance order), L_h_out [B*H] (Eq. 1) and nnz_out [1]; BSA_ECAPACITY in
+ * the device error word if nnz_out > col_cap.  workspace: >=
+ * bsa_workspace_size(plan, BSA_OP_AUGMENT) bytes, 256-aligned.
+ */
+int bsa_augment(const bsa_plan* plan, const int32_t* row_ptr, const uint16_t* order, const int32_t* extra,
+                int32_t* row_ptr_out, int32_t* col_idx_out, int64_t col_cap, float* L_h_out,
+                int64_t* nnz_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Host-only: the review's SASA budget for R ranks with workloads L_r (Eqs.
+ * 7-10): dL_r = max L - L_r; B_r = n1 * dL_r if dL_r > n2 * max L, else 0
+ * (the pages use n1 = 0.8, n2 = 0.07); L_aug_r = L_r + B_r; *A = max(0,
+ * max L_aug - max L) + S (the visible overhead).  When heads_per_rank is not
+ * NULL, extra_per_head (sum of heads_per_rank entries) receives
+ * floor(B_r / heads_per_rank[r]) for each head of rank r, in rank order -- the
+ * per-head input of bsa_augment.  Host pointers; no CUDA call.
+ */
+int bsa_sasa_budget(int R, const float* L_r, float n1, float n2, float S, float* B_r, float* L_aug, float* A,
+                    const int32_t* heads_per_rank, int32_t* extra_per_head);
+
+/*
+ * Fixed mask on the device: a local window plus rotating global anchors (the
+ * LVSA wiki page, "TL;DR" and "Key points": a structured local window pattern
+ * plus global anchor blocks that shift across diffusion timesteps; the page
+ * gives no sizes).  Row (b,h,i) keeps key block j when the latent-frame
+ * ranges of blocks i and j (frame-major token order) come within
+ * radius_frames frames, plus the anchors {(step + m*floor(nb/n_anchor)) mod
+ * nb : m < n_anchor}; columns ascending and unique, identical for every head.
+ * radius_frames >= 0, 0 <= n_anchor <= 64, step >= 0.  Outputs as for
+ * bsa_route (row_ptr [rows+1], col_idx [col_cap], nnz [1]; BSA_ECAPACITY in
+ * the device error word if nnz > col_cap).  workspace: >=
+ * bsa_workspace_size(plan, BSA_OP_MASK) bytes, 256-aligned.
+ */
+int bsa_mask_window_anchor(const bsa_plan* plan, int radius_frames, int n_anchor, int step,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, int64_t* nnz,
+                           void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Block-sparse attention (the pages' "Block-Sparse Attention Execution"):

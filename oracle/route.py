@@ -88,6 +88,7 @@ class RouteResult:
     ambiguous: np.ndarray   # bool [rows]: decision within TIE_REL of a tie / of p
     P_sorted: np.ndarray    # fp64 [rows, nb]: P in importance order
     P: np.ndarray           # fp64 [rows, nb]: P in key-block order
+    order: np.ndarray       # int64 [rows, nb]: the full key-block importance order
     qbar: np.ndarray        # fp64 [B*H, nb, d]
     kbar: np.ndarray        # fp64 [B*H, nb, d]
     scores: np.ndarray      # fp64 [B*H, nb, nb]
@@ -152,5 +153,5 @@ def route(q: np.ndarray, k: np.ndarray, T: int, Hs: int, Ws: int, block: int,
     per_head = n_i.reshape(B * H, nb).sum(axis=1)
     L_h = per_head.astype(np.float32) / np.float32(nb)
     return RouteResult(nb=nb, counts=n_i, n_p=n_p, row_ptr=row_ptr, col_idx=col_idx,
-                       L_h=L_h, nnz=int(row_ptr[-1]), ambiguous=amb, P_sorted=Ps, P=P,
+                       L_h=L_h, nnz=int(row_ptr[-1]), ambiguous=amb, P_sorted=Ps, P=P, order=order_idx,
                        qbar=qbar, kbar=kbar, scores=scores)

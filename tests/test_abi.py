@@ -92,3 +92,22 @@ def test_plan_create_without_gpu_reports_cuda_error(bsa):
     assert bsa._lib.bsa_plan_create(ctypes.byref(h), 1, 2, 4, 16, 16, 64, 64, 0) == bsa.BSA_ECUDA
     with pytest.raises(bsa.BsaError):
         bsa.Plan(1, 2, 4, 16, 16, 64, 64)
+
+
+def test_sasa_budget_host_matches_oracle(bsa):
+    """bsa_sasa_budget is host-only: Eqs. 7-10 against the oracle, and the per-head split."""
+    import numpy as np
+    import oracle.sasa as sasa
+    rng = np.random.default_rng(4)
+    for _ in range(50):
+        R = int(rng.integers(1, 9))
+        L = rng.uniform(1, 30, size=R).astype(np.float32)
+        n1, n2, S = float(rng.uniform(0, 1)), float(rng.uniform(0, 0.2)), float(rng.uniform(0, 1))
+        heads = rng.integers(1, 6, size=R)
+        B, La, A, ex = bsa.bsa_sasa_budget(L, n1, n2, S, heads)
+        ref = sasa.budget(L.astype(np.float64), np.float32(n1), np.float32(n2), np.float32(S))
+        assert np.allclose(B.numpy(), ref["B"], rtol=1e-5, atol=1e-5)
+        assert np.allclose(La.numpy(), ref["L_aug"], rtol=1e-5, atol=1e-5)
+        assert abs(A - ref["A"]) < 1e-4
+        assert list(ex.numpy()) == list(sasa.extra_per_head(B.numpy().astype(np.float64), heads))
+    assert bsa._lib.bsa_sasa_budget(0, None, 0.8, 0.07, 0.0, None, None, None, None, None) == bsa.BSA_EINVAL
