@@ -50,6 +50,8 @@ _SIGS = {
     "bsa_route_order": (_I, [_P, _P, ctypes.POINTER(_P)]),
     "bsa_augment": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
     "bsa_sasa_budget": (_I, [_I, _P, ctypes.c_float, ctypes.c_float, ctypes.c_float, _P, _P, _P, _P, _P]),
+    "bsa_rlb_plan": (_I, [_I, _I, _P, _P, _P, ctypes.POINTER(_I), _P, _P, _P]),
+    "bsa_balance_policy": (_I, [ctypes.c_float, ctypes.c_float, ctypes.c_float]),
     "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_run": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
@@ -179,6 +181,52 @@ def bsa_sasa_budget(L_r, n1=0.8, n2=0.07, S=0.0, heads_per_rank=None):
     _check(_lib.bsa_sasa_budget(R, L.data_ptr(), float(n1), float(n2), float(S), B.data_ptr(), La.data_ptr(),
                                 A.data_ptr(), _ptr(hp), _ptr(ex)), "bsa_sasa_budget")
     return B, La, float(A[0]), ex
+
+
+def bsa_rlb_plan(L_h, head_rank, R):
+    """Host-only load-balancing plan: (moves [(src, dst, head)], L_r_new, rho_before, rho_after)."""
+    Lh = torch.tensor(list(L_h), dtype=torch.float32)
+    hr = torch.tensor(list(head_rank), dtype=torch.int32)
+    moves = torch.empty(3 * R, dtype=torch.int32)
+    n = _I()
+    Ln = torch.empty(R, dtype=torch.float32)
+    rb, ra = torch.empty(1), torch.empty(1)
+    _check(_lib.bsa_rlb_plan(R, Lh.numel(), hr.data_ptr(), Lh.data_ptr(), moves.data_ptr(), ctypes.byref(n),
+                             Ln.data_ptr(), rb.data_ptr(), ra.data_ptr()), "bsa_rlb_plan")
+    mv = moves[:3 * n.value].view(-1, 3).tolist()
+    return [tuple(m) for m in mv], Ln, float(rb[0]), float(ra[0])
+
+
+def bsa_balance_policy(rho, k1=1.05, k2=1.10) -> int:
+    return _lib.bsa_balance_policy(float(rho), float(k1), float(k2))
+
+
+def migrate_heads(x, local_heads, moves, rank, group=None):
+    """Carry out a plan's head moves with torch.distributed point-to-point sends.
+
+    x: [B, N, H_local, d] tensor holding the heads listed in `local_heads`
+    (global ids, same order); moves: [(src, dst, head)] from bsa_rlb_plan.
+    Returns (x_new, local_heads_new): sent heads removed, received heads
+    appended in move order.  Plumbing only: the data leaves and arrives as is.
+    """
+    import torch.distributed as dist
+    keep = list(range(len(local_heads)))
+    recv_bufs, recv_ids, reqs = [], [], []
+    for src, dst, h in moves:
+        if src == rank:
+            i = local_heads.index(h)
+            keep.remove(i)
+            reqs.append(dist.isend(x[:, :, i].contiguous(), dst, group=group))
+        elif dst == rank:
+            buf = torch.empty_like(x[:, :, 0])
+            reqs.append(dist.irecv(buf, src, group=group))
+            recv_bufs.append(buf)
+            recv_ids.append(h)
+    for q in reqs:
+        q.wait()
+    parts = [x[:, :, i] for i in keep] + recv_bufs
+    heads = [local_heads[i] for i in keep] + recv_ids
+    return torch.stack(parts, dim=2) if parts else x[:, :, :0], heads
 
 
 def bsa_route_intermediates(plan, workspace):

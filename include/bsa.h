@@ -197,6 +197,31 @@ int bsa_sasa_budget(int R, const float* L_r, float n1, float n2, float S, float*
                     const int32_t* heads_per_rank, int32_t* extra_per_head);
 
 /*
+ * Host-only: the runtime load-balancing plan of the review (section 3 "Stage
+ * 2", Eqs. 1-6, section 3.2 and its RLB algorithm flow) for R ranks holding
+ * n_heads heads: head h lives on rank head_rank[h] and carries workload L_h[h]
+ * (Eq. 1; e.g. bsa_route's L_h, all-gathered).  A plan is a set of disjoint
+ * rank pairs, each swapping one head of each side (one send and one receive
+ * per rank, at most one local head moved); the empty plan is allowed.  The
+ * returned plan minimises (max_r L_r_new, Var_r L_r_new) lexicographically
+ * (Eq. 6) with L_r_new from Eq. 5, deterministically, so every rank computes
+ * the same plan from the same inputs.  moves: int32 [3*R] receives
+ * *n_moves triples (src rank, dst rank, head); L_r_new: float [R];
+ * rho_before / rho_after (may be NULL): Eq. 2.  R <= 12 (BSA_EUNSUPPORTED
+ * above); host pointers; no CUDA call.
+ */
+int bsa_rlb_plan(int R, int n_heads, const int32_t* head_rank, const float* L_h, int32_t* moves,
+                 int* n_moves, float* L_r_new, float* rho_before, float* rho_after);
+
+/*
+ * Host-only: the review's piecewise enabling policy (section 3.3): 0 = do
+ * nothing (rho < k1), 1 = slack augmentation only (k1 <= rho < k2), 2 = load
+ * balancing then augmentation (rho >= k2); the pages use k1 = 1.05, k2 = 1.10.
+ * Negative status for invalid arguments.
+ */
+int bsa_balance_policy(float rho, float k1, float k2);
+
+/*
  * Fixed mask on the device: a local window plus rotating global anchors (the
  * LVSA wiki page, "TL;DR" and "Key points": a structured local window pattern
  * plus global anchor blocks that shift across diffusion timesteps; the page

@@ -1,0 +1,67 @@
+"""The load-balancing flow across ranks, on CPU with gloo: every rank all-gathers
+the head workloads, plans independently and gets the same plan (no solve-and-
+broadcast), then the planned heads move by point-to-point sends."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, hpr, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import block_sparse_attention_top_b200 as bsa
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local_heads = list(range(rank * hpr, (rank + 1) * hpr))
+        g = torch.Generator().manual_seed(100 + rank)
+        L_local = torch.rand(hpr, generator=g) * 10 + (8.0 if rank == 0 else 0.0)     # rank 0 overloaded
+        gathered = [torch.empty(hpr) for _ in range(world)]
+        dist.all_gather(gathered, L_local)
+        L_h = torch.cat(gathered)
+        owner = [h // hpr for h in range(world * hpr)]
+        moves, L_new, rho_b, rho_a = bsa.bsa_rlb_plan(L_h.tolist(), owner, world)
+        # per-head payload [B=1, N=3, H_local, d=2] whose values name the head
+        x = torch.stack([torch.full((1, 3, 2), float(h)) for h in local_heads], dim=2)
+        x2, heads2 = bsa.migrate_heads(x, local_heads, moves, rank)
+        ok = all(float(x2[0, 0, i, 0]) == float(h) for i, h in enumerate(heads2))
+        q.put((rank, moves, [round(v, 5) for v in L_new.tolist()], heads2, ok, rho_b, rho_a))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,hpr", [(2, 3), (4, 5)])
+def test_all_ranks_plan_alike_and_heads_move(world, hpr):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, hpr, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {r[0]: r[1:] for r in (q.get(timeout=120) for _ in range(world))}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    plans = [res[r][0] for r in range(world)]
+    assert all(p == plans[0] for p in plans)                      # identical, independently computed
+    assert all(res[r][1] == res[0][1] for r in range(world))
+    assert all(res[r][3] for r in range(world))                   # payloads arrived intact
+    # the heads each rank holds afterwards follow the plan
+    owner = {h: h // hpr for h in range(world * hpr)}
+    for src, dst, h in plans[0]:
+        owner[h] = dst
+    for r in range(world):
+        assert sorted(res[r][2]) == sorted(h for h, o in owner.items() if o == r)
+    assert res[0][5] <= res[0][4]                                 # rho does not grow
