@@ -255,7 +255,7 @@ def run_ours(args, rank, world, local_rank):
         "route_gbs": round(rbytes / (route_avg * 1e-3) / 1e9, 1),
         "route_frac_of_hbm": round(rbytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "prepare_ms_per_call": round(statistics.mean(prep_ms), 4),
-        "roofline": {"bound": "tensor", "kernel": "k_attn_tc", "achieved": round(achieved, 2),
+        "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": round(achieved, 2),
                      "peak": pk["bf16_tflops"], "peak_kind": f"bf16 dense burst, {pk_kind}", "unit": "TFLOP/s",
                      "frac": round(achieved / pk["bf16_tflops"], 4),
                      "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
@@ -271,21 +271,31 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+ATTN_KERNEL = "k_attn_pp"        # the attention kernel bsa_attn_run launches for block 128
+ATTN_SOURCES = ("attn_pp.cu", "tc_common.cuh")
+ATTN_PROFILE = "k_attn_pp_wan21_480p.md"
+
+
+def sources_sha256(names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "block_sparse_attention_top_b200", "csrc", n), "rb").read())
+    return h.hexdigest()
+
+
 def load_traffic():
     """DRAM bytes per launch of the attention kernel, from the committed ncu summary
-    (profiles/k_attn_tc_wan21_480p.md), or None if that summary was taken on a
-    different attn_tc.cu than the one built here."""
-    import hashlib
-    src = os.path.join(ROOT, "block_sparse_attention_top_b200", "csrc", "attn_tc.cu")
-    path = os.path.join(ROOT, "profiles", "k_attn_tc_wan21_480p.md")
+    (profiles/k_attn_pp_wan21_480p.md), or None if that summary was taken on
+    different kernel sources than the ones built here."""
+    path = os.path.join(ROOT, "profiles", ATTN_PROFILE)
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
         fields = {}
         for line in open(path):
             if ":" in line and line.startswith("- "):
                 key, val = line[2:].split(":", 1)
                 fields[key.strip()] = val.strip().strip("`")
-        if fields.get("attn_tc.cu sha256") != sha:
+        if fields.get("sources sha256") != sources_sha256(ATTN_SOURCES):
             return None
         return int(fields["dram bytes per launch"].replace(",", ""))
     except Exception:

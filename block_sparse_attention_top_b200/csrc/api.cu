@@ -1,6 +1,7 @@
 // libbsa C ABI: plans, argument validation, workspace layout, stream-ordered
-// launch sequences.  Kernels live in route.cu, prepare.cu, attn_simt.cu and
-// attn_tc.cu.
+// launch sequences.  Kernels live in route.cu, route_static.cu, masks.cu,
+// augment.cu, prepare.cu, attn_pp.cu (block 128), attn_tc.cu (block 64) and
+// attn_simt.cu; balance.cu is host code.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -298,6 +299,9 @@ static int attn_run_common(const bsa_plan* p, const int32_t* row_ptr, const int3
     if (simt) {
         BSA_LAUNCH(launch_attn_simt(*p, base + L.qp, base + L.kp, base + L.vp, row_ptr, col_idx,
                                     (const int32_t*)(base + L.work), o, s));
+    } else if (attn_pp_supported(*p)) {
+        BSA_LAUNCH(launch_attn_pp(*p, base + L.qp, base + L.kp, base + L.vp, row_ptr, col_idx,
+                                  (const int32_t*)(base + L.work), o, s));
     } else {
         BSA_LAUNCH(launch_attn_tc(*p, base + L.qp, base + L.kp, base + L.vp, row_ptr, col_idx,
                                   (const int32_t*)(base + L.work), (int32_t*)(base + L.counter), o, s));

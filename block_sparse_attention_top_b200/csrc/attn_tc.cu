@@ -447,8 +447,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (!(ok = mbar_wait(bar(B_QFULL), q_it & 1, abort_flag))) break;
                 ++q_it;
                 // Q -> TMEM (16 columns of bf16 per copy), then its shared buffer is free.
-                // The previous item's QKs, issued earlier by this thread, have read the
-                // old Q columns: tensor-core operations of one thread run in issue order.
+                // The previous item's QKs have completed: the last PV issued above waited
+                // for that item's last P, which the softmax warps write only after that
+                // block's QK result arrived (a copy is not ordered behind earlier MMAs).
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)

@@ -76,6 +76,12 @@ cudaError_t launch_attn_simt(const bsa_plan& p, const void* qp, const void* kp, 
 cudaError_t launch_attn_tc(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work,
                            int32_t* counter, void* o, cudaStream_t s);
+// Ping-pong tensor-core kernel (two softmax warp groups on alternating key
+// blocks); block = 128 only, d in {64, 128}.
+bool attn_pp_supported(const bsa_plan& p);
+cudaError_t launch_attn_pp(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
+                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work, void* o,
+                           cudaStream_t s);
 
 // Host-side token order (no CUDA).
 void token_order(int T, int Hs, int Ws, int order, int32_t* perm);

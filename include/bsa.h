@@ -246,8 +246,10 @@ int bsa_mask_window_anchor(const bsa_plan* plan, int radius_frames, int n_anchor
  * token order.  Rows with no key block produce zeros.
  * q, k, v, o: bf16 [B,N,H,d]; row_ptr/col_idx: a CSR mask as above.
  * Equivalent to bsa_attn_prepare followed by bsa_attn_run on `stream`.
- * A column outside [0, nb) or a decreasing row_ptr is skipped and recorded
- * as BSA_EDEVICE in the device error word.
+ * A column outside [0, nb) is recorded as BSA_EDEVICE in the device error
+ * word and the output rows of its query block are then unspecified (every
+ * other row is still computed); a decreasing row_ptr counts as an empty row
+ * and is recorded the same way.
  * workspace: >= bsa_workspace_size(plan, BSA_OP_ATTN) bytes, 256-aligned.
  */
 int bsa_sparse_attn(const bsa_plan* plan, const void* q, const void* k, const void* v,
@@ -259,7 +261,10 @@ int bsa_sparse_attn(const bsa_plan* plan, const void* q, const void* k, const vo
  * prepare: orders the work items (b,h,i) heaviest first by their number of
  *   key blocks, and copies Q, K, V into reordered, zero-padded
  *   [B, H, nb*block, d] bf16 tiles inside the workspace.
- * run: the persistent tcgen05 attention kernel over that work list; writes O.
+ * run: the persistent tcgen05 attention kernel over that work list (for
+ *   block 128: two softmax warp groups on alternating key blocks, QK and PV
+ *   issued by separate threads; for block 64: one group splitting each row
+ *   in halves); writes O.
  * run must follow prepare on the same stream with the same workspace.
  */
 int bsa_attn_prepare(const bsa_plan* plan, const void* q, const void* k, const void* v,

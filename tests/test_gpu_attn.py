@@ -122,8 +122,9 @@ def test_identity_order_and_user_mask(bsa, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_malformed_mask_reported(bsa, kernel):
-    w = syn.workload(2, T=1, Hs=16, Ws=16, H=1, block=64)
+@pytest.mark.parametrize("block", [64, 128])
+def test_malformed_mask_reported(bsa, kernel, block):
+    w = syn.workload(2, T=1, Hs=16, Ws=block // 4, H=1, block=block)        # four query blocks
     x = syn.make_inputs(w, seed=2)
     nb = w.nb
     row_ptr = np.array([0, 2, 4, 5, 6], dtype=np.int64)
