@@ -250,15 +250,18 @@ def run_ours(args, rank, world, local_rank):
                    "density": round(float(nnz_v) / (w.rows * w.nb), 4)},
         "attn_ms_per_call": round(attn_avg, 4),
         "attn_tflops": round(achieved, 2),
-        "attn_frac_of_bf16_peak": round(achieved / pk["bf16_tflops"], 4),
+        "attn_frac_of_bf16_burst": round(achieved / pk["bf16_tflops"], 4),
         "route_ms_per_call": round(route_avg, 4),
         "route_gbs": round(rbytes / (route_avg * 1e-3) / 1e9, 1),
         "route_frac_of_hbm": round(rbytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "prepare_ms_per_call": round(statistics.mean(prep_ms), 4),
+        # the attention kernel is timed inside a ~1 s loop of steps under the power cap:
+        # the sustained bf16 peak is its denominator (the burst one is reported beside it)
         "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": round(achieved, 2),
-                     "peak": pk["bf16_tflops"], "peak_kind": f"bf16 dense burst, {pk_kind}", "unit": "TFLOP/s",
-                     "frac": round(achieved / pk["bf16_tflops"], 4),
-                     "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
+                     "peak": pk["bf16_tflops_sustained"],
+                     "peak_kind": f"bf16 dense sustained (cuBLAS 8192^3 for 4 s), {pk_kind}", "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
+                     "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
                      "traffic": traffic},
         "e2e": {"value": round(flops_sum / (e2e_ms_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms_max, 3),
