@@ -9,6 +9,10 @@ Modules:
   hilbert    frame-major 2-D Hilbert token order (enumerated curve)
   route      pooling, block scores, softmax, Top-p CDF, Top-k floor, CSR, L_h
   attention  softmax attention over the retained key blocks; dense attention
+  fp8        the same attention with an e4m3 P.V product (per-block V scales)
+  masks      window + rotating anchor block masks
+  sasa       slack-aware augmentation budget (Eqs. 7-10) and the augmented CSR
+  rlb        runtime load balancing: rank loads, rho, the pair-swap plan search
 
 Pin status: every function is pinned by tests/test_oracle_*.py against
 closed forms, invariants, brute force or a library routine (see each module's
