@@ -56,6 +56,9 @@ _SIGS = {
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_run": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_run_simt": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_sparse_attn_fp8v": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_attn_prepare_fp8v": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bsa_attn_run_fp8v": (_I, [_P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_last_device_error": (_I, [_P, _P]),
     "bsa_strerror": (ctypes.c_char_p, [_I]),
 }
@@ -256,6 +259,21 @@ def bsa_attn_run_simt(plan, row_ptr, col_idx, o, workspace, stream=None):
                                   workspace.numel(), _stream(stream))
 
 
+def bsa_sparse_attn_fp8v(plan, q, k, v, row_ptr, col_idx, o, workspace, stream=None):
+    return _lib.bsa_sparse_attn_fp8v(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx),
+                                     _ptr(o), _ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def bsa_attn_prepare_fp8v(plan, q, k, v, row_ptr, workspace, stream=None):
+    return _lib.bsa_attn_prepare_fp8v(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(workspace),
+                                      workspace.numel(), _stream(stream))
+
+
+def bsa_attn_run_fp8v(plan, row_ptr, col_idx, o, workspace, stream=None):
+    return _lib.bsa_attn_run_fp8v(plan.handle, _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+
+
 def bsa_last_device_error(plan, stream=None) -> int:
     return _lib.bsa_last_device_error(plan.handle, _stream(stream))
 
@@ -286,4 +304,13 @@ def sparse_attn(plan: Plan, q, k, v, row_ptr, col_idx, workspace=None, out=None,
         workspace = plan.workspace(BSA_OP_ATTN, q.device)
     o = torch.empty_like(q) if out is None else out
     _check(bsa_sparse_attn(plan, q, k, v, row_ptr, col_idx, o, workspace, stream), "bsa_sparse_attn")
+    return o
+
+
+def sparse_attn_fp8v(plan: Plan, q, k, v, row_ptr, col_idx, workspace=None, out=None, stream=None):
+    """As sparse_attn, with the e4m3 P.V product (block 128 only)."""
+    if workspace is None:
+        workspace = plan.workspace(BSA_OP_ATTN, q.device)
+    o = torch.empty_like(q) if out is None else out
+    _check(bsa_sparse_attn_fp8v(plan, q, k, v, row_ptr, col_idx, o, workspace, stream), "bsa_sparse_attn_fp8v")
     return o

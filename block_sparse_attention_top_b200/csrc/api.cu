@@ -75,6 +75,7 @@ AttnWs attn_ws_layout(const bsa_plan& p) {
     w.hist = off; off += align_up((size_t)(p.nb + 2) * sizeof(int32_t));
     w.bins = off; off += align_up((size_t)(p.nb + 2) * sizeof(int32_t));
     w.counter = off; off += align_up(4 * sizeof(int32_t));
+    w.vscale = off; off += align_up((size_t)p.B * p.H * p.d * sizeof(float));   // e4m3 V: per-channel scales
     w.total = off;
     return w;
 }
@@ -301,7 +302,7 @@ static int attn_run_common(const bsa_plan* p, const int32_t* row_ptr, const int3
                                     (const int32_t*)(base + L.work), o, s));
     } else if (attn_pp_supported(*p)) {
         BSA_LAUNCH(launch_attn_pp(*p, base + L.qp, base + L.kp, base + L.vp, row_ptr, col_idx,
-                                  (const int32_t*)(base + L.work), o, s));
+                                  (const int32_t*)(base + L.work), o, nullptr, s));
     } else {
         BSA_LAUNCH(launch_attn_tc(*p, base + L.qp, base + L.kp, base + L.vp, row_ptr, col_idx,
                                   (const int32_t*)(base + L.work), (int32_t*)(base + L.counter), o, s));
@@ -325,6 +326,46 @@ int bsa_sparse_attn(const bsa_plan* p, const void* q, const void* k, const void*
     if (!col_idx || !o) return BSA_EINVAL;
     if (int rc = bsa_attn_prepare(p, q, k, v, row_ptr, ws, ws_bytes, stream)) return rc;
     return bsa_attn_run(p, row_ptr, col_idx, o, ws, ws_bytes, stream);
+}
+
+// ---- FP8 (e4m3) P.V product ----
+int bsa_attn_prepare_fp8v(const bsa_plan* p, const void* q, const void* k, const void* v,
+                          const int32_t* row_ptr, void* ws, size_t ws_bytes, void* stream) {
+    if (!p || !q || !k || !v || !row_ptr) return BSA_EINVAL;
+    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(row_ptr, 4))
+        return BSA_EINVAL;
+    if (!attn_pp_supported(*p)) return BSA_EUNSUPPORTED;
+    const AttnWs L = attn_ws_layout(*p);
+    if (int rc = check_ws(ws, ws_bytes, L.total)) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* base = (char*)ws;
+    BSA_LAUNCH(launch_worklist(*p, row_ptr, (int32_t*)(base + L.hist), (int32_t*)(base + L.bins),
+                               (int32_t*)(base + L.work), s));
+    BSA_LAUNCH(launch_permute(*p, q, k, v, base + L.qp, base + L.kp, nullptr, s, 2));
+    BSA_LAUNCH(launch_quant_v(*p, v, (float*)(base + L.vscale), base + L.vp, s));
+    return BSA_OK;
+}
+
+int bsa_attn_run_fp8v(const bsa_plan* p, const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                      void* ws, size_t ws_bytes, void* stream) {
+    if (!p || !row_ptr || !col_idx || !o) return BSA_EINVAL;
+    if (misaligned(o, 16) || misaligned(row_ptr, 4) || misaligned(col_idx, 4)) return BSA_EINVAL;
+    if (!attn_pp_supported(*p)) return BSA_EUNSUPPORTED;
+    const AttnWs L = attn_ws_layout(*p);
+    if (int rc = check_ws(ws, ws_bytes, L.total)) return rc;
+    char* base = (char*)ws;
+    BSA_LAUNCH(launch_attn_pp(*p, base + L.qp, base + L.kp, base + L.vp, row_ptr, col_idx,
+                              (const int32_t*)(base + L.work), o, (const float*)(base + L.vscale),
+                              (cudaStream_t)stream));
+    return BSA_OK;
+}
+
+int bsa_sparse_attn_fp8v(const bsa_plan* p, const void* q, const void* k, const void* v,
+                         const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                         void* ws, size_t ws_bytes, void* stream) {
+    if (!col_idx || !o) return BSA_EINVAL;
+    if (int rc = bsa_attn_prepare_fp8v(p, q, k, v, row_ptr, ws, ws_bytes, stream)) return rc;
+    return bsa_attn_run_fp8v(p, row_ptr, col_idx, o, ws, ws_bytes, stream);
 }
 
 int bsa_last_device_error(const bsa_plan* p, void* stream) {

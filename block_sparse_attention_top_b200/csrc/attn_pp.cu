@@ -49,11 +49,19 @@
 // A column outside [0, nb) is recorded as BSA_EDEVICE and replaced by the
 // nearest valid block, so every role still walks the same sequence.
 //
+// FP8 variant (F8 = true; the review's V quantization, format not stated):
+// V arrives as e4m3 tiles [d x 128 keys] per (head, key block) with per-
+// channel scales sigma_c (quant.cu); the probabilities enter as e4m3(16 P)
+// with P relative to the running maximum, which is rescaled once it grows by
+// more than 2^4 (so 16 P <= 256 fits e4m3), PV is a kind::f8f6f4 MMA with
+// fp32 accumulation, and the epilogue writes O[:, c] * sigma_c / l.
+//
 // Every wait on an mbarrier spins on test_wait and is bounded (about 4 s); on
 // expiry the CTA records BSA_EDEVICE, raises a shared abort flag that stops
 // the other roles, drains its own tensor-core work and frees TMEM.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "bsa_internal.cuh"
 #include "tc_common.cuh"
@@ -74,15 +82,16 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kPolyPairs = 0;             // pairs in every 8 exponentiated on the FMA pipe (0: all on
                                           // MUFU; 1 and 2 measured slower in this kernel)
 
-template <int D>
+template <int D, bool F8>
 struct PPLayout {
     static constexpr uint32_t kColP = kColO + D;            // P0; P1 follows
     static_assert(kColP + 2 * (kBlk / 2) <= kTmemCols, "TMEM budget");
     static constexpr int kTile = kBlk * D * 2;      // one Q, K or V tile: D/64 slabs of [128 rows x 128 B]
+    static constexpr int kVTile = F8 ? D * 128 : kTile;   // e4m3 V: [D rows x 128 B] (keys along a row)
     static constexpr int offQ = 0;
     static constexpr int offK = offQ + kTile;
     static constexpr int offV = offK + kKStages * kTile;
-    static constexpr int offPub = offV + kVStages * kTile;   // float m[2][128], l[2][128]
+    static constexpr int offPub = offV + kVStages * kVTile;  // float m[2][128], l[2][128]
     static constexpr int offBar = offPub + 4 * kBlk * 4;
     static constexpr int kBars = 40;
     static constexpr int offMisc = offBar + kBars * 8;
@@ -106,6 +115,7 @@ struct Params {
     int N, H, nb, rows;
     int64_t npad;
     float scale_log2;
+    const float* sigma;      // F8: per (head, channel) V scale, [B*H, D]
 };
 
 __device__ __forceinline__ int item_index(int k, int cta, int grid) {
@@ -160,11 +170,34 @@ __device__ __forceinline__ float softmax_row(const uint32_t* s, float scale, flo
     return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-template <int D>
+// The same for the FP8 product: p (already in units of 16 P) rounded to e4m3,
+// four keys to a 32-bit word (key 4w in the low byte), and the row sum.
+template <int N, bool RAGGED>
+__device__ __forceinline__ float softmax_row_e4m3(const uint32_t* s, float scale, float neg_m, uint32_t* pk) {
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+#pragma unroll
+    for (int c = 0; c < N; c += 4) {
+        float x0, x1, x2, x3;
+        ffma2(x0, x1, __uint_as_float(s[c]), __uint_as_float(s[c + 1]), scale, scale, neg_m, neg_m);
+        ffma2(x2, x3, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]), scale, scale, neg_m, neg_m);
+        const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1), p2 = ex2_mufu(x2), p3 = ex2_mufu(x3);
+        const int u = (c / 4) & 3;
+        fadd2(acc[2 * u], acc[2 * u + 1], acc[2 * u], acc[2 * u + 1], p0, p1);
+        fadd2(acc[2 * u], acc[2 * u + 1], acc[2 * u], acc[2 * u + 1], p2, p3);
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
+        pk[c / 4] = lo | (hi << 16);
+    }
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const Params prm) {
-    using L = PPLayout<D>;
+    using L = PPLayout<D, F8>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -234,10 +267,16 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int st = u % kVStages;
                     const uint32_t use = u / kVStages;
                     if (use > 0 && !(ok = mbar_wait(bar(V_EMPTY0 + st), (use - 1) & 1, abort_flag))) break;
-                    mbar_expect_tx(bar(V_FULL0 + st), L::kTile);
-                    for (int s = 0; s < D / 64; ++s)
-                        tma_load_2d(sbase + L::offV + st * L::kTile + s * kBlk * 128, &tmV, s * 64, y,
+                    mbar_expect_tx(bar(V_FULL0 + st), L::kVTile);
+                    if constexpr (F8) {
+                        // e4m3 tile of (head, block j): rows (bh * nb + j) * D .. + D, 128 keys each
+                        tma_load_2d(sbase + L::offV + st * L::kVTile, &tmV, 0, (int)(((int64_t)bh * nb + j) * D),
                                     bar(V_FULL0 + st));
+                    } else {
+                        for (int s = 0; s < D / 64; ++s)
+                            tma_load_2d(sbase + L::offV + st * L::kVTile + s * kBlk * 128, &tmV, s * 64, y,
+                                        bar(V_FULL0 + st));
+                    }
                 }
             }
             if (!ok) { *abort_flag = 1; record_error(prm.err, BSA_EDEVICE, -1); }
@@ -283,7 +322,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     } else if (warp == kPvWarp) {
         // ---------------------------------------------------------- PV issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_pv = instr_desc(D, 1);
+            constexpr uint32_t idesc_pv = F8 ? instr_desc_e4m3(D) : instr_desc(D, 1);
             Walk pc;
             uint32_t up = 0;
             bool ok = true;
@@ -297,11 +336,20 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (!(ok = mbar_wait(bar(V_FULL0 + st), (up / kVStages) & 1, abort_flag))) break;
                 fence_after();
                 const bool fresh = pc.first();
+                const uint32_t p_tmem = tmem + L::kColP + (up & 1) * (kBlk / 2);
+                if constexpr (F8) {
+                    // K = 32 keys (32 bytes) per MMA: P columns kk*8.., V row bytes kk*32..
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t b = smem_desc(sbase + L::offV + st * L::kTile + kk * 16 * 128, kBlk * 128, 1024);
-                    mma_ts(tmem + kColO, tmem + L::kColP + (up & 1) * (kBlk / 2) + kk * 8, b, idesc_pv,
-                           (fresh && kk == 0) ? 0u : 1u);
+                    for (int kk = 0; kk < kBlk / 32; ++kk) {
+                        const uint64_t b = smem_desc(sbase + L::offV + st * L::kVTile + kk * 32, 16, 1024);
+                        mma_ts_f8(tmem + kColO, p_tmem + kk * 8, b, idesc_pv, (fresh && kk == 0) ? 0u : 1u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const uint64_t b = smem_desc(sbase + L::offV + st * L::kVTile + kk * 16 * 128, kBlk * 128, 1024);
+                        mma_ts(tmem + kColO, p_tmem + kk * 8, b, idesc_pv, (fresh && kk == 0) ? 0u : 1u);
+                    }
                 }
                 commit(bar(PV_DONE0 + (up & 1)));
                 commit(bar(V_EMPTY0 + st));
@@ -372,14 +420,20 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 bool rescale = false;
                 if (first) {
                     m_use = mx;
-                } else if (mx > m_prev + 8.f) {
+                } else if (mx > m_prev + (F8 ? 4.f : 8.f)) {
                     alpha = ex2_mufu(m_prev - mx);
                     m_use = mx;
                     rescale = true;
                 }
                 uint32_t pk[kBlk / 2];
-                const float rowsum = ragged ? softmax_row<kBlk, true>(sv, prm.scale_log2, -m_use, pk)
-                                            : softmax_row<kBlk, false>(sv, prm.scale_log2, -m_use, pk);
+                float rowsum;
+                if constexpr (F8) {                          // in units of 16 P: 2^(s*scale - m + 4)
+                    rowsum = ragged ? softmax_row_e4m3<kBlk, true>(sv, prm.scale_log2, 4.f - m_use, pk)
+                                    : softmax_row_e4m3<kBlk, false>(sv, prm.scale_log2, 4.f - m_use, pk);
+                } else {
+                    rowsum = ragged ? softmax_row<kBlk, true>(sv, prm.scale_log2, -m_use, pk)
+                                    : softmax_row<kBlk, false>(sv, prm.scale_log2, -m_use, pk);
+                }
                 m_pub[mine] = m_use;                         // the other group's next block may start
                 mbar_arrive(bar(M_PUB0 + pub_mine));
                 // PV_{t-2} done: this group's P buffer is free.  PVs of odd and even
@@ -407,8 +461,9 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                         tmem_st32(tmem + lane_base + kColO + c * 32, o);
                     }
                 }
+                constexpr int kPCols = F8 ? kBlk / 4 : kBlk / 2;     // 32-bit TMEM columns of one P row
 #pragma unroll
-                for (int c = 0; c < kBlk / 64; ++c)
+                for (int c = 0; c < kPCols / 32; ++c)
                     tmem_st32(tmem + lane_base + L::kColP + g * (kBlk / 2) + c * 32, pk + 32 * c);
                 // running row sum
                 float l_prev = 0.f;
@@ -433,6 +488,11 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + kColO + c * 32, o);
                     tmem_wait_ld();
+                    if constexpr (F8) {                      // per-channel V scale
+                        const float* sg = prm.sigma + (int64_t)(r / nb) * D + c * 32;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * __ldg(sg + e));
+                    }
                     if (row_real) {
 #pragma unroll
                         for (int e = 0; e < 32; e += 8) {
@@ -460,19 +520,20 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     }
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
                    cudaStream_t s) {
-    using L = PPLayout<D>;
+    using L = PPLayout<D, F8>;
     const int64_t rows_total = (int64_t)p.B * p.H * p.nb * p.block;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, qp, rows_total, D, kBlk) || !make_map(&mk, kp, rows_total, D, kBlk) ||
-        !make_map(&mv, vp, rows_total, D, kBlk))
+    if (!make_map(&mq, qp, rows_total, D, kBlk) || !make_map(&mk, kp, rows_total, D, kBlk))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_attn_pp<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (F8 ? !make_map_u8(&mv, vp, (int64_t)p.B * p.H * p.nb * D, D) : !make_map(&mv, vp, rows_total, D, kBlk))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_attn_pp<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<int64_t>(p.num_sms, p.rows);
-    k_attn_pp<D><<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, prm);
+    k_attn_pp<D, F8><<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, prm);
     return cudaGetLastError();
 }
 
@@ -482,7 +543,7 @@ bool attn_pp_supported(const bsa_plan& p) { return p.block == kBlk && (p.d == 12
 
 cudaError_t launch_attn_pp(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work, void* o,
-                           cudaStream_t s) {
+                           const float* sigma, cudaStream_t s) {
     Params prm;
     prm.row_ptr = row_ptr;
     prm.col_idx = col_idx;
@@ -496,8 +557,13 @@ cudaError_t launch_attn_pp(const bsa_plan& p, const void* qp, const void* kp, co
     prm.rows = (int)p.rows;
     prm.npad = p.nb * p.block;
     prm.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
-    if (p.d == 128) return launch<128>(p, qp, kp, vp, prm, s);
-    return launch<64>(p, qp, kp, vp, prm, s);
+    prm.sigma = sigma;
+    if (sigma) {                      // e4m3 V tiles at vp, scales at sigma
+        if (p.d == 128) return launch<128, true>(p, qp, kp, vp, prm, s);
+        return launch<64, true>(p, qp, kp, vp, prm, s);
+    }
+    if (p.d == 128) return launch<128, false>(p, qp, kp, vp, prm, s);
+    return launch<64, false>(p, qp, kp, vp, prm, s);
 }
 
 }  // namespace bsa

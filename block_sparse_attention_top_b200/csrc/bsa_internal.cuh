@@ -34,7 +34,7 @@ RouteWs route_ws_layout(const bsa_plan& p);
 inline size_t mask_ws_bytes(const bsa_plan& p) { return align_up((size_t)p.rows * sizeof(int32_t)); }
 
 struct AttnWs {
-    size_t qp, kp, vp, work, hist, bins, counter, total;
+    size_t qp, kp, vp, work, hist, bins, counter, vscale, total;
 };
 AttnWs attn_ws_layout(const bsa_plan& p);
 
@@ -68,8 +68,9 @@ cudaError_t launch_augment(const bsa_plan& p, const int32_t* row_ptr, const uint
 
 cudaError_t launch_worklist(const bsa_plan& p, const int32_t* row_ptr, int32_t* hist,
                             int32_t* bins, int32_t* work, cudaStream_t s);
+// n_tensors = 3: Q, K and V; 2: Q and K only (V goes through launch_quant_v)
 cudaError_t launch_permute(const bsa_plan& p, const void* q, const void* k, const void* v,
-                           void* qp, void* kp, void* vp, cudaStream_t s);
+                           void* qp, void* kp, void* vp, cudaStream_t s, int n_tensors = 3);
 cudaError_t launch_attn_simt(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
                              const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work,
                              void* o, cudaStream_t s);
@@ -79,9 +80,13 @@ cudaError_t launch_attn_tc(const bsa_plan& p, const void* qp, const void* kp, co
 // Ping-pong tensor-core kernel (two softmax warp groups on alternating key
 // blocks); block = 128 only, d in {64, 128}.
 bool attn_pp_supported(const bsa_plan& p);
+// sigma != null: vp holds e4m3 V tiles from launch_quant_v and sigma their
+// per-(head, channel) scales (the FP8 P.V product).
 cudaError_t launch_attn_pp(const bsa_plan& p, const void* qp, const void* kp, const void* vp,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work, void* o,
-                           cudaStream_t s);
+                           const float* sigma, cudaStream_t s);
+// e4m3 V: sigma [B*H*d] floats (per head and channel), vt [B*H*nb*d, 128] bytes
+cudaError_t launch_quant_v(const bsa_plan& p, const void* v, float* sigma, void* vt, cudaStream_t s);
 
 // Host-side token order (no CUDA).
 void token_order(int T, int Hs, int Ws, int order, int32_t* perm);

@@ -105,7 +105,7 @@ cudaError_t launch_worklist(const bsa_plan& p, const int32_t* row_ptr, int32_t* 
 }
 
 cudaError_t launch_permute(const bsa_plan& p, const void* q, const void* k, const void* v, void* qp,
-                           void* kp, void* vp, cudaStream_t s) {
+                           void* kp, void* vp, cudaStream_t s, int n_tensors) {
     const int vec_per_row = p.d * 2 / 16;
     const int64_t npad = p.nb * p.block;
     const int64_t total = (int64_t)p.B * npad * p.H * vec_per_row;
@@ -113,7 +113,7 @@ cudaError_t launch_permute(const bsa_plan& p, const void* q, const void* k, cons
     int64_t blocks = (total + t - 1) / t;
     const int64_t cap = (int64_t)p.num_sms * 16;
     if (blocks > cap) blocks = cap;
-    dim3 grid((unsigned)blocks, 3);
+    dim3 grid((unsigned)blocks, (unsigned)n_tensors);
     k_permute<<<grid, t, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (uint4*)qp, (uint4*)kp,
                                  (uint4*)vp, p.d_perm, (int)p.N, p.H, vec_per_row, npad, total);
     return cudaGetLastError();

@@ -273,6 +273,30 @@ int bsa_attn_run(const bsa_plan* plan, const int32_t* row_ptr, const int32_t* co
                  void* o, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Block-sparse attention with an FP8 P.V product (the review's section 3
+ * "Block-Sparse Attention Execution" and section 3.4 quantize V before
+ * attention; the format is not stated).  Q.K^T stays bf16.  V of each head
+ * is scaled per channel, sigma_c = amax over the N tokens of |V[:, c]| / 448,
+ * and rounded to e4m3 (OCP E4M3, nearest-even, saturating); the softmax
+ * probabilities enter the product as e4m3(16 P) with P taken relative to a
+ * running maximum that lags the true one by less than 2^4; products are
+ * summed in fp32 and output column c is scaled by sigma_c.  Expected error
+ * against exact attention: about 3 % mean relative (two roundings of 2^-4
+ * relative each); the tests hold it to 6 %.
+ * Same arguments, layouts and error behaviour as bsa_sparse_attn; block 128
+ * only (BSA_EUNSUPPORTED otherwise).  The e4m3 V tiles and the scales live in
+ * the attention workspace: run_fp8v must follow prepare_fp8v on the same
+ * workspace (bsa_attn_run after prepare_fp8v reads them as bf16: undefined).
+ */
+int bsa_sparse_attn_fp8v(const bsa_plan* plan, const void* q, const void* k, const void* v,
+                         const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                         void* workspace, size_t ws_bytes, void* stream);
+int bsa_attn_prepare_fp8v(const bsa_plan* plan, const void* q, const void* k, const void* v,
+                          const int32_t* row_ptr, void* workspace, size_t ws_bytes, void* stream);
+int bsa_attn_run_fp8v(const bsa_plan* plan, const int32_t* row_ptr, const int32_t* col_idx,
+                      void* o, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Same contract as bsa_attn_run, computed by a slow CUDA-core kernel (one
  * warp per query token, fp32 online softmax).  A cross-check for the
  * tensor-core kernel in tests; not a performance path.

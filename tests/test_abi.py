@@ -24,7 +24,7 @@ def bsa():
 def declared_symbols():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(bsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_symbols_exported(bsa):

@@ -1,0 +1,144 @@
+"""GPU block-sparse attention with the e4m3 P.V product against the exact
+oracle and the FP8 oracle (oracle/fp8.py), under the stated FP8 tolerance:
+mean relative error <= 6e-2 (two e4m3 roundings of 2^-4 relative each)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import oracle.fp8 as f8
+import synthetic as syn
+from _gpu import bf16_to_f64, to_dev
+from _parity import sample_blocks
+
+pytestmark = pytest.mark.gpu
+
+MEAN_REL_FP8 = 6e-2
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    from block_sparse_attention_top_b200 import build
+    build.build()
+    import block_sparse_attention_top_b200 as m
+    return m
+
+
+def mean_rel(got, want):
+    return float(np.abs(got - want).sum() / max(np.abs(want).sum(), 1e-30))
+
+
+def run_fp8(bsa, w, x, row_ptr, col_idx):
+    plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    rp = torch.from_numpy(np.asarray(row_ptr, dtype=np.int32)).cuda()
+    ci = torch.from_numpy(np.asarray(col_idx, dtype=np.int32)).cuda()
+    ws = plan.workspace(bsa.BSA_OP_ATTN)
+    o = torch.full_like(q, float("nan"))
+    assert bsa.bsa_sparse_attn_fp8v(plan, q, k, v, rp, ci, o, ws) == 0
+    assert bsa.bsa_last_device_error(plan) == 0
+    return o, ws, plan
+
+
+def _al(x):
+    return (x + 255) // 256 * 256
+
+
+def ws_views(w, ws):
+    """The e4m3 V tiles and the per-channel scales inside the attention workspace."""
+    tile = w.B * w.H * w.nb * w.block * w.d * 2
+    off_v = 2 * _al(tile)
+    off = 3 * _al(tile)
+    off += _al(w.rows * 4) + 2 * _al((w.nb + 2) * 4) + _al(16)
+    vt = ws[off_v:off_v + w.B * w.H * w.nb * w.d * 128].cpu().numpy()
+    sigma = ws[off:off + 4 * w.B * w.H * w.d].view(torch.float32).cpu().numpy()
+    return vt, sigma
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=2, Hs=33, Ws=17, H=2, d=64, block=128),
+    dict(T=3, Hs=16, Ws=16, H=2, d=128, block=128),
+    dict(T=4, Hs=30, Ws=52, H=2, d=128, block=128),
+])
+@pytest.mark.parametrize("p", [0.6, 1.0])
+def test_small_shapes_full(bsa, shape, p):
+    w = syn.workload(2, **shape)
+    x = syn.make_inputs(w, seed=31)
+    m = oracle.route(x["q"], x["k"], w.T, w.Hs, w.Ws, w.block, p, 1)
+    o, ws, _ = run_fp8(bsa, w, x, m.row_ptr, m.col_idx)
+    got = bf16_to_f64(o)
+    exact = oracle.sparse_attention(x["q"], x["k"], x["v"], w.T, w.Hs, w.Ws, w.block, m.row_ptr, m.col_idx)
+    emul = f8.sparse_attention_fp8v(x["q"], x["k"], x["v"], w.T, w.Hs, w.Ws, w.block, m.row_ptr, m.col_idx)
+    e_gpu, e_orc = mean_rel(got, exact), mean_rel(emul, exact)
+    print(f"fp8 mean rel vs exact: gpu {e_gpu:.4f}, oracle {e_orc:.4f}; gpu vs oracle {mean_rel(got, emul):.4f}")
+    assert np.isfinite(got).all()
+    assert e_gpu <= MEAN_REL_FP8 and mean_rel(got, emul) <= MEAN_REL_FP8
+    # the same quantization scheme: the GPU's error is the oracle's, not a different one
+    assert 0.5 * e_orc <= e_gpu <= 2.0 * e_orc
+
+
+def test_quantized_v_and_scales(bsa):
+    """sigma_c exactly fl32(amax / 448); the e4m3 tiles equal the oracle's rounding of
+    V / sigma except at rounding ties decided differently by fp32 and fp64."""
+    w = syn.workload(2, T=3, Hs=16, Ws=16, H=2, d=128, block=128)
+    x = syn.make_inputs(w, seed=32)
+    m = oracle.route(x["q"], x["k"], w.T, w.Hs, w.Ws, w.block, 0.9, 1)
+    _, ws, _ = run_fp8(bsa, w, x, m.row_ptr, m.col_idx)
+    vt, sigma = ws_views(w, ws)
+    perm = oracle.token_perm(w.T, w.Hs, w.Ws)
+    table = f8.e4m3_table()
+    mismatch = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            vh = oracle.decode(x["v"][b, :, h, :])
+            want_sigma = f8.channel_scales(vh).astype(np.float32)
+            bh = b * w.H + h
+            np.testing.assert_array_equal(sigma[bh * w.d:(bh + 1) * w.d], want_sigma)
+            for j in range(w.nb):
+                toks = perm[j * w.block:min(w.N, (j + 1) * w.block)]
+                want = np.zeros((w.d, 128))
+                want[:, :len(toks)] = f8.round_e4m3(vh[toks] / want_sigma.astype(np.float64)).T
+                base = (bh * w.nb + j) * w.d * 128
+                got = table[vt[base:base + w.d * 128]].reshape(w.d, 128)
+                diff = got != want
+                mismatch += int(diff.sum())
+                if diff.any():   # any disagreement is one grid step at a near-tie
+                    a, bb = np.abs(got[diff]), np.abs(want[diff])
+                    assert np.all(np.abs(a - bb) <= 0.125 * np.maximum(a, bb) + 2.0 ** -9)
+    assert mismatch <= 1e-3 * w.B * w.H * w.nb * w.d * 128
+
+
+@pytest.mark.parametrize("cid,p_index", [(2, 0), (3, 1)])
+def test_full_size_sampled(bsa, cid, p_index):
+    w = syn.workload(cid)
+    x = syn.make_inputs(w, seed=syn.seed_for(cid, p_index))
+    m = oracle.route(x["q"], x["k"], w.T, w.Hs, w.Ws, w.block, w.ps[p_index], w.k_floor)
+    o, _, _ = run_fp8(bsa, w, x, m.row_ptr, m.col_idx)
+    perm = oracle.token_perm(w.T, w.Hs, w.Ws)
+    counts = np.diff(m.row_ptr)
+    rows = sample_blocks(counts, w.B * w.H, w.nb, 48, seed=cid)
+    got, exact, emul = [], [], []
+    for r in rows:
+        bh, i = divmod(int(r), w.nb)
+        b, h = divmod(bh, w.H)
+        toks = perm[i * w.block:min(w.N, (i + 1) * w.block)]
+        got.append(bf16_to_f64(o[b, torch.from_numpy(toks).cuda(), h, :]))
+        exact.append(oracle.attend_block(x["q"], x["k"], x["v"], perm, w.block, m.row_ptr, m.col_idx, w.H, b, h, i))
+        emul.append(f8.attend_block_fp8v(x["q"], x["k"], x["v"], perm, w.block, m.row_ptr, m.col_idx, w.H, b, h, i))
+    got, exact, emul = (np.concatenate(a) for a in (got, exact, emul))
+    e_gpu, e_orc = mean_rel(got, exact), mean_rel(emul, exact)
+    print(f"config {cid}: fp8 mean rel vs exact gpu {e_gpu:.4f} oracle {e_orc:.4f}")
+    assert e_gpu <= MEAN_REL_FP8
+    assert 0.5 * e_orc <= e_gpu <= 2.0 * e_orc
+
+
+def test_block_64_unsupported(bsa):
+    w = syn.workload(2, T=1, Hs=16, Ws=16, H=1, block=64)
+    plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block)
+    x = syn.make_inputs(w, seed=1)
+    q = to_dev(x["q"])
+    rp = torch.zeros(w.rows + 1, dtype=torch.int32, device="cuda")
+    ci = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = plan.workspace(bsa.BSA_OP_ATTN)
+    o = torch.empty_like(q)
+    assert bsa.bsa_sparse_attn_fp8v(plan, q, q, q, rp, ci, o, ws) == bsa.BSA_EUNSUPPORTED
