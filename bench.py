@@ -193,6 +193,27 @@ def run_ours(args, rank, world, local_rank):
     attn_ms = [e[2].elapsed_time(e[3]) for e in events]
     total_ms = sum(step_ms)
 
+    # the FP8 P.V variant on the same inputs and mask (reported beside the bf16 headline)
+    fp8_steps = max(3, min(args.steps, 50))
+    fp8_prep, fp8_run = [], []
+    for i in range(fp8_steps + 2):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        rc = bsa.bsa_attn_prepare_fp8v(plan, q, k, v, row_ptr, ws_attn, stream)
+        ev[1].record(stream)
+        rc |= bsa.bsa_attn_run_fp8v(plan, row_ptr, col_idx, o, ws_attn, stream)
+        ev[2].record(stream)
+        if rc:
+            raise RuntimeError(f"fp8 attention call failed: {rc}")
+        if i >= 2:
+            fp8_prep.append(ev)
+    torch.cuda.synchronize()
+    if bsa.bsa_last_device_error(plan) != 0:
+        raise RuntimeError("device error in the fp8 variant")
+    fp8_prep_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in fp8_prep)
+    fp8_run_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in fp8_prep)
+
     # end to end through the public API with pinned host buffers
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -266,6 +287,10 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(flops_sum / (e2e_ms_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms_max, 3),
                 "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2},
+        "attn_fp8v": {"kernel": ATTN_KERNEL + "<F8>", "calls": fp8_steps, "attn_ms_per_call": round(fp8_run_ms, 4),
+                      "tflops": round(flops / (fp8_run_ms * 1e-3) / 1e12, 2),
+                      "prepare_ms_per_call": round(fp8_prep_ms, 4),
+                      "note": "Q.K^T bf16, P.V e4m3 (per-channel V scales); same FLOP count as the bf16 path"},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
     }
