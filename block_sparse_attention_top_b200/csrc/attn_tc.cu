@@ -39,9 +39,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "bsa_internal.cuh"
+#include "tc_common.cuh"
 
 namespace bsa {
 namespace {
@@ -53,201 +52,8 @@ constexpr int kVWarp = 2 + kSoftmaxWarps;
 constexpr int kTileM = 128;                          // query rows per tile (TMEM lanes)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColQ = 384;
-constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
-// ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ unsigned long long globaltimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// Non-blocking probe of a phase.  The suspending try_wait form was measured to
-// wake up late (about 1000 cycles after the phase completed), which sat on
-// the critical path of every handshake; the waits below spin on test_wait.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    const unsigned long long t0 = globaltimer();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_test(bar, parity)) return true;
-        if ((n & 1023u) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > kTimeoutNs) return false;
-        }
-    }
-}
-// Bounded wait: false if the abort flag is raised or the time limit passes.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, abort_flag);
-}
-// Warp-uniform bounded wait (every lane polls; all lanes agree on the outcome).
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-// 128 rows x 256 bits from shared memory (matrix descriptor) into TMEM lanes 0..127
-__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
-    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-#define BSA_R8(b) "=r"(r[b + 0]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), \
-                  "=r"(r[b + 4]), "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7])
-#define BSA_W8(b) "r"(r[b + 0]), "r"(r[b + 1]), "r"(r[b + 2]), "r"(r[b + 3]), \
-                  "r"(r[b + 4]), "r"(r[b + 5]), "r"(r[b + 6]), "r"(r[b + 7])
-// 32 lanes x 32 consecutive 32-bit columns
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : BSA_R8(0), BSA_R8(8), BSA_R8(16), BSA_R8(24)
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), BSA_W8(0), BSA_W8(8), BSA_W8(16), BSA_W8(24)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-        ::"r"(taddr), BSA_W8(0), BSA_W8(8)
-        : "memory");
-}
-#undef BSA_R8
-#undef BSA_W8
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 format (version 1).
-// lbo / sbo in bytes.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128,
-// A K-major; B K-major (0) or MN-major (1).
-__host__ __device__ constexpr uint32_t instr_desc(int n, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) |
-           ((uint32_t)(kTileM >> 4) << 24);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-__device__ __forceinline__ float ex2_mufu(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-    float y;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
-    return y;
-}
-
-// Packed fp32 pairs (sm_100 f32x2 instructions): d = a * b + c, d = a + b.
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
-                                      float c1) {
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-// 2^x for a pair of values on the FMA pipe for x in [-127, 128): split x = j + f with j = rint(x),
-// f in [-1/2, 1/2] (adding 1.5 * 2^23 rounds to an integer held in the low
-// mantissa bits), a degree-3 polynomial for 2^f (coefficients from a
-// relative-error minimax fit on [-1/2, 1/2], max relative error 7.5e-5), and
-// j added straight into the exponent field.  Accurate far beyond the bf16
-// rounding P receives.
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
-    x0 = fmaxf(x0, -127.f);
-    x1 = fmaxf(x1, -127.f);
-    float t0, t1, j0, j1, f0, f1, p0, p1;
-    fadd2(t0, t1, x0, x1, 12582912.f, 12582912.f);
-    fadd2(j0, j1, t0, t1, -12582912.f, -12582912.f);
-    ffma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);
-    ffma2(p0, p1, 0.0551716648f, 0.0551716648f, f0, f1, 0.2426111251f, 0.2426111251f);
-    ffma2(p0, p1, p0, p1, f0, f1, 0.6932609677f, 0.6932609677f);
-    ffma2(p0, p1, p0, p1, f0, f1, 0.9999280572f, 0.9999280572f);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
-// Maximum of n values with 8 independent chains (n a multiple of 16).
-template <int n>
-__device__ __forceinline__ float row_max(const uint32_t* v, float init) {
-    float m[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) m[u] = max3(init, __uint_as_float(v[2 * u]), __uint_as_float(v[2 * u + 1]));
-#pragma unroll
-    for (int c = 16; c < n; c += 16)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) m[u] = max3(m[u], __uint_as_float(v[c + 2 * u]), __uint_as_float(v[c + 2 * u + 1]));
-    return fmaxf(fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5])), fmaxf(m[6], m[7]));
-}
+using namespace tc;
 
 // P for this warp's half row: p = 2^(s * scale - m), packed to bf16 pairs, and
 // the half-row sum.  One pair in eight goes through the FMA-pipe polynomial
@@ -351,9 +157,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    tc_fence_before();
+    fence_before();
     __syncthreads();
-    tc_fence_after();
+    fence_after();
     const uint32_t tmem = *tmem_slot;
 
     const int grid = gridDim.x, cta = blockIdx.x;
@@ -426,15 +232,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (!mbar_wait(bar(B_PFULL), pv_it & 1, abort_flag)) return false;
                 const int st = it % kVStages;
                 if (!mbar_wait(bar(B_VFULL0 + st), (it / kVStages) & 1, abort_flag)) return false;
-                tc_fence_after();
+                fence_after();
                 const uint32_t p_tmem = tmem + ((it & 1) ? kColS1 : kColS0);   // P overwrote S(it)
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
                     const uint64_t b = smem_desc(sbase + L::offV + st * L::kKV + kk * 16 * 128, BLK * 128, 1024);
-                    tc_mma_ts(tmem + kColO, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                    mma_ts(tmem + kColO, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
                 }
-                tc_commit(bar(B_PVDONE));
-                tc_commit(bar(B_VEMPTY0 + st));
+                commit(bar(B_PVDONE));
+                commit(bar(B_VEMPTY0 + st));
                 ++pv_it;
                 return true;
             };
@@ -450,12 +256,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // The previous item's QKs have completed: the last PV issued above waited
                 // for that item's last P, which the softmax warps write only after that
                 // block's QK result arrived (a copy is not ordered behind earlier MMAs).
-                tc_fence_after();
+                fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc_cp_128x256b(tmem + kColQ + kk * 8,
+                    cp_128x256b(tmem + kColQ + kk * 8,
                                    smem_desc(sbase + L::offQ + (kk / 4) * kTileM * 128 + (kk % 4) * 32, 16, 1024));
-                tc_commit(bar(B_QEMPTY));
+                commit(bar(B_QEMPTY));
                 int local = 0;
                 int jn = prm.col_idx[beg];
                 for (int jj = beg; jj < end && ok; ++jj) {
@@ -467,15 +273,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     // P_FULL arrival this thread waited on for PV(kv_it-2), and that PV, which
                     // read P from the same columns, was issued earlier by this thread.
                     if (!(ok = mbar_wait(bar(B_KFULL0 + st), (kv_it / kKStages) & 1, abort_flag))) break;
-                    tc_fence_after();
+                    fence_after();
                     const uint32_t d_s = tmem + ((kv_it & 1) ? kColS1 : kColS0);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t b = smem_desc(sbase + L::offK + st * L::kKV + (kk / 4) * BLK * 128 + (kk % 4) * 32, 16, 1024);
-                        tc_mma_ts(d_s, tmem + kColQ + kk * 8, b, idesc_qk, kk > 0 ? 1u : 0u);
+                        mma_ts(d_s, tmem + kColQ + kk * 8, b, idesc_qk, kk > 0 ? 1u : 0u);
                     }
-                    tc_commit(bar(B_SFULL0 + (kv_it & 1)));
-                    tc_commit(bar(B_KEMPTY0 + st));
+                    commit(bar(B_SFULL0 + (kv_it & 1)));
+                    commit(bar(B_KEMPTY0 + st));
                     if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
                     ++kv_it;
                     ++local;
@@ -488,7 +294,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 record_error(prm.err, BSA_EDEVICE, -2);
             }
             // drain: everything this thread issued completes before TMEM is freed
-            tc_commit(bar(B_DRAIN));
+            commit(bar(B_DRAIN));
             volatile int no_abort = 0;
             mbar_wait(bar(B_DRAIN), 0, &no_abort);
         }
@@ -521,7 +327,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const int sb = kv_it & 1;
                 const uint32_t s_col = sb ? kColS1 : kColS0;
                 if (!(ok = warp_wait(bar(B_SFULL0 + sb), (kv_it >> 1) & 1, abort_flag))) break;
-                tc_fence_after();
+                fence_after();
                 // padding keys of a ragged last block
                 const int valid_keys = prm.N - j * BLK;
                 const bool ragged = valid_keys < BLK;
@@ -569,7 +375,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (local > 0) {
                     if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
                     ++pv_it;
-                    tc_fence_after();
+                    fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                         for (int c = 0; c < OC / 32; ++c) {
@@ -583,7 +389,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                 }
                 tmem_wait_st();
-                tc_fence_before();
+                fence_before();
                 mbar_arrive(bar(B_PFULL));
                 ++kv_it;
                 ++local;
@@ -598,7 +404,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             // memory (slots alternate by item; a bounded mbarrier pairs the two warps)
             if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
             ++pv_it;
-            tc_fence_after();
+            fence_after();
             float* ls = xchg + 4 * kTileM + (items & 1) * 2 * kTileM;
             ls[half * kTileM + row] = l;
             mbar_arrive(bar(B_PAIR0 + quad));
@@ -623,46 +429,20 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                 }
             }
-            tc_fence_before();
+            fence_before();
         }
         if (!ok) { *abort_flag = 1; record_error(prm.err, BSA_EDEVICE, -3); }
     }
 
-    tc_fence_before();
+    fence_before();
     __syncthreads();
-    tc_fence_after();
+    fence_after();
     if (warp == 1) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
 // ----------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// [rows, d] bf16 row-major, box = [box_rows, 64] with 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1u, 1u};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int BLK>
 cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
                    cudaStream_t s) {
