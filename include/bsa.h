@@ -11,7 +11,11 @@
  *     blocks); the workload L_h is the review's Eq. 1;
  *   - attention: FVAttn review, section 3 "Block-Sparse Attention Execution"
  *     (attention over the retained blocks, then head-order / token-order
- *     restoration).
+ *     restoration), in bf16 or with the review's V quantization (section
+ *     3.4) read as an e4m3 P.V product;
+ *   - around them: the SASA augmentation (section 3 "Stage 3", Eqs. 7-10),
+ *     the runtime load-balancing planner (section 3 "Stage 2", Eqs. 1-6) and
+ *     a window + rotating-anchor mask producer (the LVSA wiki page).
  *
  * Conventions shared by every call
  *   - Q, K, V, O: [B, N, H, d] row-major (d fastest), N = T*Hs*Ws tokens in
@@ -99,8 +103,9 @@ int bsa_plan_info(const bsa_plan* plan, int64_t* N, int64_t* nb, int64_t* rows);
 int bsa_token_order(int T, int Hs, int Ws, int order, int32_t* perm);
 
 /* Bytes of device workspace that bsa_route (BSA_OP_ROUTE), bsa_sparse_attn
- * (BSA_OP_ATTN), bsa_mask_window_anchor (BSA_OP_MASK) or
- * bsa_augment (BSA_OP_AUGMENT); 0 for a NULL plan or unknown op. */
+ * and bsa_sparse_attn_fp8v (BSA_OP_ATTN), bsa_mask_window_anchor
+ * (BSA_OP_MASK) or bsa_augment (BSA_OP_AUGMENT) need; 0 for a NULL plan or
+ * an unknown op. */
 size_t bsa_workspace_size(const bsa_plan* plan, int op);
 
 /*
