@@ -51,6 +51,8 @@ _SIGS = {
     "bsa_augment": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
     "bsa_sasa_budget": (_I, [_I, _P, ctypes.c_float, ctypes.c_float, ctypes.c_float, _P, _P, _P, _P, _P]),
     "bsa_rlb_plan": (_I, [_I, _I, _P, _P, _P, ctypes.POINTER(_I), _P, _P, _P]),
+    "bsa_rlb_gain": (_I, [_I, _P, _P, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                          _P, _P]),
     "bsa_balance_policy": (_I, [ctypes.c_float, ctypes.c_float, ctypes.c_float]),
     "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -198,6 +200,18 @@ def bsa_rlb_plan(L_h, head_rank, R):
                              Ln.data_ptr(), rb.data_ptr(), ra.data_ptr()), "bsa_rlb_plan")
     mv = moves[:3 * n.value].view(-1, 3).tolist()
     return [tuple(m) for m in mv], Ln, float(rb[0]), float(ra[0])
+
+
+def bsa_rlb_gain(L_r, L_r_new, c, P=0.0, C=0.0, A=0.0):
+    """(K, G) of the review's gain model (Eqs. 3-4, 11) for rank loads before and after a plan."""
+    a = torch.tensor([float(v) for v in L_r], dtype=torch.float32)
+    b = torch.tensor([float(v) for v in L_r_new], dtype=torch.float32)
+    if a.shape != b.shape:
+        raise ValueError("L_r and L_r_new must have the same length")
+    K, G = ctypes.c_double(), ctypes.c_double()
+    _check(_lib.bsa_rlb_gain(a.numel(), a.data_ptr(), b.data_ptr(), float(c), float(P), float(C), float(A),
+                             ctypes.byref(K), ctypes.byref(G)), "bsa_rlb_gain")
+    return K.value, G.value
 
 
 def bsa_balance_policy(rho, k1=1.05, k2=1.10) -> int:

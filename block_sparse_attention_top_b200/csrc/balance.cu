@@ -142,6 +142,20 @@ int bsa_rlb_plan(int R, int n_heads, const int32_t* head_rank, const float* L_h,
     return BSA_OK;
 }
 
+int bsa_rlb_gain(int R, const float* L_r, const float* L_r_new, double c, double P, double C, double A,
+                 double* K, double* G) {
+    if (R < 1 || !L_r || !L_r_new || !K || !G) return BSA_EINVAL;
+    double before = -INFINITY, after = -INFINITY;
+    for (int r = 0; r < R; ++r) {
+        if (!(L_r[r] >= 0.0f) || !(L_r_new[r] >= 0.0f)) return BSA_EINVAL;
+        before = std::max(before, (double)L_r[r]);
+        after = std::max(after, (double)L_r_new[r]);
+    }
+    *K = c * (before - after);
+    *G = *K - P - C - A;
+    return BSA_OK;
+}
+
 int bsa_balance_policy(float rho, float k1, float k2) {
     if (!(rho >= 0.0f) || !(k1 <= k2)) return BSA_EINVAL;
     return rho < k1 ? 0 : (rho < k2 ? 1 : 2);

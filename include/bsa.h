@@ -219,6 +219,19 @@ int bsa_rlb_plan(int R, int n_heads, const int32_t* head_rank, const float* L_h,
                  int* n_moves, float* L_r_new, float* rho_before, float* rho_after);
 
 /*
+ * Host-only: the review's gain model for a migration plan (section 3 "Stage
+ * 2", Eqs. 3-4, and the joint form of Eq. 11): the straggler time saved
+ * K = c * (max_r L_r - max_r L_r_new), with c the time per unit of workload,
+ * and the net gain G = K - P - C - A, with P the plan-search time, C the
+ * communication time of the migration and A the slack-augmentation cost (0
+ * without augmentation; the pages give no values for c, P, C or A).  L_r,
+ * L_r_new: [R] host arrays (e.g. from bsa_rlb_plan).  Negative status for
+ * R < 1, null pointers or negative loads.
+ */
+int bsa_rlb_gain(int R, const float* L_r, const float* L_r_new, double c, double P, double C, double A,
+                 double* K, double* G);
+
+/*
  * Host-only: the review's piecewise enabling policy (section 3.3): 0 = do
  * nothing (rho < k1), 1 = slack augmentation only (k1 <= rho < k2), 2 = load
  * balancing then augmentation (rho >= k2); the pages use k1 = 1.05, k2 = 1.10.

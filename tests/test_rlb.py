@@ -67,3 +67,19 @@ def test_planner_errors_and_policy(bsa):
     for rho in (1.0, 1.049, 1.05, 1.099, 1.1, 1.34):
         assert bsa.bsa_balance_policy(rho) == orlb.policy(rho)
     assert bsa.bsa_balance_policy(1.2, 1.2, 1.1) == bsa.BSA_EINVAL
+
+
+def test_gain_model_matches_oracle(bsa):
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        R = int(rng.integers(1, 9))
+        L = rng.uniform(0, 20, R).astype(np.float32)
+        Ln = rng.uniform(0, 20, R).astype(np.float32)
+        c, P, C = (float(v) for v in rng.uniform(0, 3, 3))
+        K, G = bsa.bsa_rlb_gain(L, Ln, c, P, C)
+        Ko, Go = orlb.gain(L.astype(np.float64), Ln.astype(np.float64), c=c, P=P, C=C)
+        assert K == pytest.approx(Ko, rel=1e-12, abs=1e-12) and G == pytest.approx(Go, rel=1e-12, abs=1e-12)
+        # the joint model of Eq. 11 subtracts the augmentation cost A as well
+        assert bsa.bsa_rlb_gain(L, Ln, c, P, C, A=0.25)[1] == pytest.approx(Go - 0.25, abs=1e-12)
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_rlb_gain([1.0, -2.0], [1.0, 1.0], 1.0)
