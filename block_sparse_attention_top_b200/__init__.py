@@ -6,8 +6,17 @@ library is missing the import fails loudly; there is no CPU path.
 
 The functions keep the C names (bsa_route, bsa_sparse_attn, ...) and take
 torch tensors where the C call takes device pointers; `Plan` wraps
-bsa_plan_create / bsa_plan_destroy.  `route` and `sparse_attn` are thin
-conveniences that allocate the outputs and the workspace with torch.
+bsa_plan_create / bsa_plan_destroy.  `route`, `sparse_attn` and
+`sparse_attn_fp8v` are thin conveniences that allocate the outputs and the
+workspace with torch.
+
+    import torch, block_sparse_attention_top_b200 as bsa
+    # q, k, v: bf16 [B, N, H, d] on cuda, N = T * Hs * Ws latent tokens
+    plan = bsa.Plan(B, H, T, Hs, Ws, d, 128)             # frame-major Hilbert order
+    row_ptr, col_idx, L_h, nnz = bsa.route(plan, q, k, 0.9, 4)   # Top-p 0.9, floor 4
+    o = bsa.sparse_attn(plan, q, k, v, row_ptr, col_idx)        # bf16 [B, N, H, d]
+    o8 = bsa.sparse_attn_fp8v(plan, q, k, v, row_ptr, col_idx)  # e4m3 P.V product
+    assert bsa.bsa_last_device_error(plan) == bsa.BSA_OK
 """
 from __future__ import annotations
 
