@@ -391,7 +391,7 @@ def reference_step(x, w, p, full_flops, rng):
     return (t1 - t0) * w.B * w.H + (t2 - t1) * full_flops / fl
 
 
-def run_reference(args):
+def run_reference(args, world=1):
     """The fp64 CPU oracle on bounded samples of the same workload (the reference arm)."""
     w = syn.workload(CID)
     p = w.ps[P_INDEX]
@@ -407,7 +407,7 @@ def run_reference(args):
     value = full_flops / (ms * 1e-3) / 1e12
     sample = (f"each step: oracle routing of 1 random head (of {w.H}) and attention on 1 random query block of "
               f"it, timed and extrapolated linearly to the full step ({w.H} heads, {full_flops / 1e12:.2f} TFLOP)")
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_desc(w), "global_batch": w.B, "seq_len": w.N,
@@ -431,7 +431,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
     if world > 1:
         import datetime
