@@ -82,6 +82,13 @@ def test_null_plan_calls(bsa):
     assert bsa._lib.bsa_workspace_size(None, 0) == 0
     assert bsa._lib.bsa_route(None, None, None, 0, 0.9, 1, None, None, 0, None, None, None, 0, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_sparse_attn(None, None, None, None, None, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_sparse_attn_fp8v(None, None, None, None, None, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_attn_prepare_fp8v(None, None, None, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_attn_run_fp8v(None, None, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_attn_prepare(None, None, None, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_attn_run(None, None, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_augment(None, None, None, None, None, None, 0, None, None, None, 0, None) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_mask_window_anchor(None, 2, 8, 0, None, None, 0, None, None, 0, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_last_device_error(None, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_plan_info(None, None, None, None) == bsa.BSA_EINVAL
 
