@@ -11,6 +11,7 @@ Modules:
   attention  softmax attention over the retained key blocks; dense attention
   fp8        the same attention with an e4m3 P.V product (per-block V scales)
   masks      window + rotating anchor block masks
+  stripes    periodic diagonal stripe block masks (six parameters per head)
   sasa       slack-aware augmentation budget (Eqs. 7-10) and the augmented CSR
   rlb        runtime load balancing: rank loads, rho, the pair-swap plan search
 
