@@ -62,6 +62,7 @@ _SIGS = {
     "bsa_rlb_plan": (_I, [_I, _I, _P, _P, _P, ctypes.POINTER(_I), _P, _P, _P]),
     "bsa_rlb_gain": (_I, [_I, _P, _P, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                           _P, _P]),
+    "bsa_mask_stripes": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I64, _P]),
     "bsa_balance_policy": (_I, [ctypes.c_float, ctypes.c_float, ctypes.c_float]),
     "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -221,6 +222,23 @@ def bsa_rlb_gain(L_r, L_r_new, c, P=0.0, C=0.0, A=0.0):
     _check(_lib.bsa_rlb_gain(a.numel(), a.data_ptr(), b.data_ptr(), float(c), float(P), float(C), float(A),
                              ctypes.byref(K), ctypes.byref(G)), "bsa_rlb_gain")
     return K.value, G.value
+
+
+def bsa_mask_stripes(B, H, T, Hs, Ws, block, params, order=0):
+    """Host stripe-mask CSR (row_ptr, col_idx) as int32 CPU tensors; params: H rows of
+    (w_t, o_t, s_t, w_s, o_s, s_s)."""
+    pr = torch.tensor([[int(v) for v in row] for row in params], dtype=torch.int32).reshape(-1)
+    if pr.numel() != 6 * H:
+        raise ValueError("params must hold 6 values per head")
+    nb = -(-(T * Hs * Ws) // block)
+    rows = B * H * nb
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32)
+    nnz = ctypes.c_int64()
+    cap = rows * nb                                   # every block kept: cannot overflow
+    col_idx = torch.empty(max(cap, 1), dtype=torch.int32)
+    _check(_lib.bsa_mask_stripes(B, H, T, Hs, Ws, block, order, pr.data_ptr(), row_ptr.data_ptr(),
+                                 col_idx.data_ptr(), cap, ctypes.byref(nnz)), "bsa_mask_stripes")
+    return row_ptr, col_idx[:nnz.value].clone()
 
 
 def bsa_balance_policy(rho, k1=1.05, k2=1.10) -> int:

@@ -257,6 +257,27 @@ int bsa_mask_window_anchor(const bsa_plan* plan, int radius_frames, int n_anchor
                            void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Host-only: periodic diagonal stripe block masks (PSA pages: section 3.1,
+ * section 3.2, appendix C.2 and appendix D: per-head masks of an inter-frame
+ * and an intra-frame stripe family, each with a width, an offset and a
+ * stride, an infinite stride being a single diagonal, applied per block).
+ * params: host int32 [H][6] = (w_t, o_t, s_t, w_s, o_s, s_s): half-width
+ * (>= 0), offset and stride (<= 0: infinite) over latent-frame offsets and
+ * over row offsets inside a frame.  A family keeps key offset delta (key
+ * minus query) when |delta - o - n*s| <= w for some integer n; query block i
+ * and key block j (blocks of `order`, see bsa_plan_create) are kept together
+ * when the inter-frame family keeps some frame offset between their frame
+ * ranges and the intra-frame family some row offset between their row ranges.
+ * Outputs in HOST memory, rows r = (b*H + h)*nb + i as for bsa_route:
+ * row_ptr int32 [B*H*nb+1], col_idx int32 [col_cap] (columns ascending),
+ * nnz = the full count; BSA_ECAPACITY (columns past col_cap dropped) if nnz
+ * > col_cap.  block 64 or 128.  No CUDA call; upload the CSR for
+ * bsa_sparse_attn.
+ */
+int bsa_mask_stripes(int B, int H, int T, int Hs, int Ws, int block, int order, const int32_t* params,
+                     int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, int64_t* nnz);
+
+/*
  * Block-sparse attention (the pages' "Block-Sparse Attention Execution"):
  *   O[b, n, h, :] = sum over the real tokens t of the key blocks listed in
  *   row (b,h,i) of softmax_t(Q[b,n,h,:] . K[b,t,h,:] / sqrt(d)) V[b,t,h,:]
