@@ -122,6 +122,28 @@ def test_identity_order_and_user_mask(bsa, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+def test_stripe_mask(bsa, kernel):
+    """A PSA stripe mask from the host producer (every-other-frame stripes of
+    half-width 1 frame, rows within 4 of the query's) through the attention."""
+    w = syn.workload(2, T=6, Hs=12, Ws=16, H=2, block=128)
+    x = syn.make_inputs(w, seed=9)
+    params = [(1, 0, 2, 4, 0, 0), (0, 1, 0, w.Hs, 0, 0)]
+    rp, ci = bsa.bsa_mask_stripes(w.B, w.H, w.T, w.Hs, w.Ws, w.block, params)
+    row_ptr, col_idx = rp.numpy().astype(np.int64), ci.numpy().astype(np.int64)
+    o, status = gpu_attn(bsa, w, x["q"], x["k"], x["v"], row_ptr, col_idx, kernel)
+    assert status == 0
+    counts = np.diff(row_ptr)
+    keep = [r for r in range(w.rows) if counts[r] > 0]
+    compare_rows(o, oracle_rows(w, x["q"], x["k"], x["v"], row_ptr, col_idx, keep))
+    for r in range(w.rows):                      # rows without a key block are zeros
+        if counts[r] == 0:
+            bh, i = divmod(r, w.nb)
+            b, h = divmod(bh, w.H)
+            toks = oracle.token_perm(w.T, w.Hs, w.Ws)[i * w.block:min(w.N, (i + 1) * w.block)]
+            assert torch.all(o[b, torch.from_numpy(toks).cuda(), h, :] == 0)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("block", [64, 128])
 def test_malformed_mask_reported(bsa, kernel, block):
     w = syn.workload(2, T=1, Hs=16, Ws=block // 4, H=1, block=block)        # four query blocks
