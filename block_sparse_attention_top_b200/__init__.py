@@ -273,6 +273,55 @@ def migrate_heads(x, local_heads, moves, rank, group=None):
     return torch.stack(parts, dim=2) if parts else x[:, :, :0], heads
 
 
+def balance_step(L_h_local, local_heads, tensors, rank, world, group=None, k1=1.05, k2=1.10, n1=0.8, n2=0.07):
+    """One step of the pages' runtime balancing across ranks (FVAttn review, section 3 "Stage 2" and
+    "Stage 3", section 3.3): all-gather the per-head workloads L_h (Eq. 1), take rho (Eq. 2) and the
+    enabling policy; at policy 2 every rank computes the same pair-swap plan (Eqs. 5-6, bsa_rlb_plan)
+    and the planned heads move with point-to-point sends; at policy >= 1 the slack-augmentation budget
+    (Eqs. 7-10, bsa_sasa_budget) becomes a_h extra blocks for every query block of each local head.
+
+    L_h_local: workloads of `local_heads` (global head ids, same order); tensors: [B, N, H_local, d]
+    tensors holding those heads (all migrated alike).  Host plumbing over the library's host calls and
+    torch.distributed; nothing here computes on the device.
+    Returns dict(policy, rho_before, rho_after, moves, L_r, L_r_new, tensors, local_heads, extra).
+    """
+    import torch.distributed as dist
+    mine = (list(local_heads), [float(v) for v in L_h_local])
+    every = [None] * world
+    dist.all_gather_object(every, mine, group=group)
+    n_heads = sum(len(hs) for hs, _ in every)
+    owner, L_h = [0] * n_heads, [0.0] * n_heads
+    for r, (hs, ls) in enumerate(every):
+        for h, l in zip(hs, ls):
+            owner[h], L_h[h] = r, l
+    L_r = [sum(ls) for _, ls in every]
+    rho = max(L_r) / (sum(L_r) / world) if sum(L_r) > 0 else 1.0
+    policy = bsa_balance_policy(rho, k1, k2)
+    moves, L_r_new, rho_after = [], list(L_r), rho
+    heads = list(local_heads)
+    if policy == 2:
+        moves, L_new, _, rho_after = bsa_rlb_plan(L_h, owner, world)
+        L_r_new = L_new.tolist()
+        out = []
+        for x in tensors:
+            x_new, heads_new = migrate_heads(x, list(local_heads), moves, rank, group)
+            out.append(x_new)
+        tensors = out
+        if tensors:
+            heads = heads_new
+        else:                                             # no payload: the head list still follows the plan
+            heads = [h for h in local_heads if not any(m[2] == h and m[0] == rank for m in moves)]
+            heads += [m[2] for m in moves if m[1] == rank]
+    extra = [0] * len(heads)
+    if policy >= 1:
+        counts = [len(hs) for hs, _ in every]
+        _, _, _, ex = bsa_sasa_budget(L_r_new, n1, n2, heads_per_rank=counts)
+        lo = sum(counts[:rank])
+        extra = ex[lo:lo + counts[rank]].tolist()
+    return dict(policy=policy, rho_before=rho, rho_after=rho_after, moves=moves, L_r=L_r, L_r_new=L_r_new,
+                tensors=tensors, local_heads=heads, extra=extra)
+
+
 def bsa_route_intermediates(plan, workspace):
     a, b, c = _P(), _P(), _P()
     _check(_lib.bsa_route_intermediates(plan.handle, _ptr(workspace), ctypes.byref(a), ctypes.byref(b),

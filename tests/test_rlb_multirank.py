@@ -65,3 +65,61 @@ def test_all_ranks_plan_alike_and_heads_move(world, hpr):
     for r in range(world):
         assert sorted(res[r][2]) == sorted(h for h, o in owner.items() if o == r)
     assert res[0][5] <= res[0][4]                                 # rho does not grow
+
+
+def _step_worker(rank, world, port, hpr, skew, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import block_sparse_attention_top_b200 as bsa
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        heads = list(range(rank * hpr, (rank + 1) * hpr))
+        g = torch.Generator().manual_seed(7 + rank)
+        L = (torch.rand(hpr, generator=g) * 4 + 10 + (skew if rank == 0 else 0.0)).tolist()
+        x = torch.stack([torch.full((1, 2, 3), float(h)) for h in heads], dim=2)
+        res = bsa.balance_step(L, heads, [x], rank, world)
+        xs = res["tensors"][0]
+        intact = all(float(xs[0, 0, i, 0]) == float(h) for i, h in enumerate(res["local_heads"]))
+        q.put((rank, res["policy"], res["moves"], res["local_heads"], res["extra"], res["L_r_new"], intact,
+               res["rho_before"], res["rho_after"]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,hpr,skew,policy", [(2, 3, 30.0, 2), (4, 2, 40.0, 2), (4, 2, 0.0, None)])
+def test_balance_step(world, hpr, skew, policy):
+    """The whole runtime flow: every rank reaches the same decision; heads and payloads follow the
+    plan; the augmentation extras are the oracle's for the post-migration loads."""
+    import oracle.rlb as orlb
+    import oracle.sasa as osasa
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_step_worker, args=(r, world, port, hpr, skew, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {r[0]: r[1:] for r in (q.get(timeout=120) for _ in range(world))}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    pol, moves = res[0][0], res[0][1]
+    assert all(res[r][0] == pol and res[r][1] == moves for r in range(world))
+    assert pol == orlb.policy(res[0][6])
+    if policy is not None:
+        assert pol == policy and moves and res[0][7] < res[0][6]
+    assert all(res[r][5] for r in range(world))                  # payloads intact
+    owner = {h: h // hpr for h in range(world * hpr)}
+    for src, dst, h in moves:
+        owner[h] = dst
+    for r in range(world):
+        assert sorted(res[r][2]) == sorted(h for h, o in owner.items() if o == r)
+    if pol >= 1:
+        B = osasa.budget(res[0][4])["B"]
+        want = osasa.extra_per_head(B, [hpr] * world)
+        got = [e for r in range(world) for e in res[r][3]]
+        assert got == list(want)
+    else:
+        assert all(all(e == 0 for e in res[r][3]) for r in range(world))
