@@ -1,19 +1,26 @@
 """Benchmark: Top-p block routing + block-sparse attention on B200.
 
-One step = one pass of the whole hot path over the 480p Wan2.1-shaped workload
-(B1 H12 d128, 21x30x52 = 32760 tokens, block 128, p = 0.9, k_floor = 4):
+One step = one pass of the whole hot path over the 720p Wan2.2-shaped workload
+(B1 H40 d128, 21x45x80 = 75600 tokens, block 128, p = 0.9, k_floor = 4):
 bsa_route (gather + mean-pool, block scores, row routing, CSR) then
-bsa_attn_prepare (heaviest-first work list, reordered Q/K/V tiles) then
-bsa_attn_run (persistent tcgen05 attention, output scattered to token order).
+bsa_attn_prepare (work list, reordered Q/K/V tiles) then bsa_attn_run
+(persistent tcgen05 attention, output scattered to token order).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--config C] [--p-index I] [--no-extras]
 
 Prints one JSON line on rank 0.  `value` is effective TFLOP/s over the whole
 step: retained-block attention FLOPs (sum over kept (row, block) pairs of
 4 * m_i * m_j * d with the real token counts) of all ranks / max-over-ranks step
-time.  N > 1 (torchrun) runs one independent replica per GPU (weak scaling, no
-collective on the data path).  `--impl reference` times the fp64 CPU oracle on a
-bounded sample of the same workload and extrapolates to the same unit.
+time.  The line also carries the attention kernel alone against the measured
+bf16 burst peak (`roofline`), routing GB/s against measured HBM, the other
+full-size workloads (480p, the skewed 720p with the three work-list
+schedules and their per-CTA imbalance, the long fixed-mask video) under
+`extra`, the FP8 P.V variant, an end-to-end figure with host buffers and the
+oracle timed on the host cores.  N > 1 (torchrun) runs one independent replica
+per GPU (weak scaling, no collective on the data path).  `--impl reference`
+times the fp64 CPU oracle on a bounded sample of the same workload and
+extrapolates to the same unit.
 """
 from __future__ import annotations
 
@@ -32,11 +39,14 @@ sys.path.insert(0, ROOT)
 
 import synthetic as syn  # noqa: E402
 
-CID = 2
-P_INDEX = 0
+CID = 3            # headline: Wan2.2-14B-shaped 720p
+P_INDEX = 1        # p = 0.9
+EXTRAS = ((2, 0), (4, 0), (5, None))     # 480p p=0.9, skewed 720p p=0.95, long fixed mask
 METRIC = "block-sparse attn ms/call & effective TFLOP/s (% bf16 peak); routing GB/s"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 10   # route: 5, prepare: 4 (hist, bins, scatter, permute), run: 1
+# route: 5 (pool, scores, row routing, scan, fill); prepare: 5 (group rank, hist, bins,
+# scatter, permute); run: 1
+KERNELS_PER_STEP = 11
 
 
 def peaks():
@@ -49,9 +59,13 @@ def peaks():
         return dict(FALLBACK), "fallback"
 
 
-def workload_desc(w):
+def workload_desc(w, p_index=None):
+    if p_index is None:
+        tail = "fixed window (+-2 latent frames) + 8 anchor blocks mask, no routing"
+    else:
+        tail = f"p={w.ps[p_index]}, k_floor={w.k_floor}"
     return (f"{w.name} (config {w.cid}): B{w.B} H{w.H} d{w.d} T{w.T}x{w.Hs}x{w.Ws}={w.N} tokens, "
-            f"block {w.block}, p={w.ps[P_INDEX]}, k_floor={w.k_floor}")
+            f"block {w.block}, {tail}")
 
 
 def attention_flops(row_ptr, col_idx, w):
@@ -121,43 +135,156 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- ours
+ATTN_KERNEL = "k_attn_pp"        # the attention kernel bsa_attn_run launches for block 128
+ATTN_SOURCES = ("attn_pp.cu", "tc_common.cuh")
+# DRAM bytes (read + write) of one k_attn_pp launch on the headline workload, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the sha256 of
+# the kernel sources it was taken on; a kernel built from other sources reports null.
+ATTN_TRAFFIC = {}
+SCHEDULES = (("l2_heads", 0), ("heaviest_first", 1), ("in_order", 2))
+
+
+def sources_sha256(names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "block_sparse_attention_top_b200", "csrc", n), "rb").read())
+    return h.hexdigest()
+
+
+class Case:
+    """One workload resident on the device: inputs, plan, mask buffers, workspaces."""
+
+    def __init__(self, bsa, torch, dev, cid, p_index, rank=0):
+        self.bsa, self.torch, self.dev = bsa, torch, dev
+        self.w = w = syn.workload(cid)
+        self.p_index = p_index
+        self.p = w.ps[p_index] if p_index is not None else None
+        seed = syn.seed_for(cid, p_index or 0) + 7919 * rank
+        self.x = syn.make_inputs(w, seed=seed)
+
+        def to_dev(a):
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+        self.q, self.k, self.v = (to_dev(self.x[n]) for n in "qkv")
+        self.plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block)
+        self.col_cap = self.plan.rows * self.plan.nb
+        self.row_ptr = torch.empty(self.plan.rows + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(self.col_cap, dtype=torch.int32, device=dev)
+        self.L_h = torch.empty(w.B * w.H, dtype=torch.float32, device=dev)
+        self.nnz = torch.empty(1, dtype=torch.int64, device=dev)
+        self.ws_route = self.plan.workspace(bsa.BSA_OP_ROUTE if self.p is not None else bsa.BSA_OP_MASK, dev)
+        self.ws_attn = self.plan.workspace(bsa.BSA_OP_ATTN, dev)
+        self.o = torch.empty_like(self.q)
+
+    def mask(self, stream):
+        """Routing (or the fixed window + anchor mask of the long workload, made on the device)."""
+        bsa, w = self.bsa, self.w
+        if self.p is None:
+            return bsa.bsa_mask_window_anchor(self.plan, 2, 8, 0, self.row_ptr, self.col_idx, self.col_cap, self.nnz,
+                                              self.ws_route, stream)
+        return bsa.bsa_route(self.plan, self.q, self.k, bsa.BSA_BF16, self.p, w.k_floor, self.row_ptr, self.col_idx,
+                             self.col_cap, self.L_h, self.nnz, self.ws_route, stream)
+
+    def prepare(self, stream):
+        return self.bsa.bsa_attn_prepare(self.plan, self.q, self.k, self.v, self.row_ptr, self.ws_attn, stream)
+
+    def run(self, stream):
+        return self.bsa.bsa_attn_run(self.plan, self.row_ptr, self.col_idx, self.o, self.ws_attn, stream)
+
+    def flops(self):
+        return attention_flops(self.row_ptr.cpu().numpy(), self.col_idx.cpu().numpy(), self.w)
+
+    def density(self):
+        return float(int(self.nnz.item())) / (self.w.rows * self.w.nb)
+
+    def route_bytes(self):
+        return route_bytes(self.w, int(self.nnz.item()), self.q.numel() * 2)
+
+    def balance(self):
+        """Per-CTA imbalance of the prepared work list (max / mean key blocks per CTA)."""
+        wptr, _, _ = self.bsa.bsa_attn_intermediates(self.plan, self.ws_attn)
+        off = wptr - self.ws_attn.data_ptr()
+        work = self.ws_attn[off:off + 4 * self.plan.rows].view(self.torch.int32).cpu()
+        rho, mx, mean = self.bsa.bsa_schedule_balance(self.plan, self.row_ptr.cpu(), work)
+        return {"rho_cta": round(rho, 4), "max_blocks_per_cta": mx, "mean_blocks_per_cta": round(mean, 1)}
+
+
+def timed_calls(torch, stream, flush, fn, n, warm=3):
+    """Mean CUDA-event time (ms) of fn(stream) over n calls, L2 flushed before each."""
+    for _ in range(warm):
+        flush.zero_()
+        fn(stream)
+    evs = []
+    for _ in range(n):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        rc = fn(stream)
+        e[1].record(stream)
+        if rc:
+            raise RuntimeError(f"bsa call failed: {rc}")
+        evs.append(e)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def extra_case(bsa, torch, dev, stream, flush, cid, p_index, n, pk):
+    """Attention (and routing) of another full-size workload, timed alone."""
+    c = Case(bsa, torch, dev, cid, p_index)
+    route_ms = timed_calls(torch, stream, flush, c.mask, n)
+    if c.prepare(stream):
+        raise RuntimeError("prepare failed")
+    fl = c.flops()
+    out = {"workload": workload_desc(c.w, p_index), "density": round(c.density(), 4)}
+    if c.p is not None:
+        rb = c.route_bytes()
+        out.update({"route_ms_per_call": round(route_ms, 4), "route_gbs": round(rb / (route_ms * 1e-3) / 1e9, 1),
+                    "route_frac_of_hbm": round(rb / (route_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    else:
+        out["mask_ms_per_call"] = round(route_ms, 4)
+    schedules = SCHEDULES if cid == 4 else SCHEDULES[:1]
+    for name, sched in schedules:
+        c.plan.set_schedule(sched)
+        if c.prepare(stream):
+            raise RuntimeError("prepare failed")
+        ms = timed_calls(torch, stream, flush, c.run, n)
+        tf = fl / (ms * 1e-3) / 1e12
+        entry = {"attn_ms_per_call": round(ms, 4), "attn_tflops": round(tf, 2),
+                 "attn_frac_of_bf16_burst": round(tf / pk["bf16_tflops"], 4)}
+        entry.update(c.balance())
+        if len(schedules) == 1:
+            out.update(entry)
+        else:
+            out.setdefault("schedules", {})[name] = entry
+            if sched == 0:
+                out.update(entry)
+    if bsa.bsa_last_device_error(c.plan) != 0:
+        raise RuntimeError(f"device error on config {cid}")
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import block_sparse_attention_top_b200 as bsa
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = syn.workload(CID)
-    p = w.ps[P_INDEX]
-    x = syn.make_inputs(w, seed=syn.seed_for(CID, P_INDEX) + 7919 * rank)
-
-    def to_dev(a):
-        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-
-    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
-    plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block)
-    col_cap = plan.rows * plan.nb
-    row_ptr = torch.empty(plan.rows + 1, dtype=torch.int32, device=dev)
-    col_idx = torch.empty(col_cap, dtype=torch.int32, device=dev)
-    L_h = torch.empty(w.B * w.H, dtype=torch.float32, device=dev)
-    nnz = torch.empty(1, dtype=torch.int64, device=dev)
-    ws_route = plan.workspace(bsa.BSA_OP_ROUTE, dev)
-    ws_attn = plan.workspace(bsa.BSA_OP_ATTN, dev)
-    o = torch.empty_like(q)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)     # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)     # > 126 MB L2
+    c = Case(bsa, torch, dev, args.config, args.p_index, rank)
+    w, p, plan = c.w, c.p, c.plan
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        rc = bsa.bsa_route(plan, q, k, bsa.BSA_BF16, p, w.k_floor, row_ptr, col_idx, col_cap, L_h, nnz, ws_route,
-                           stream)
+        rc = c.mask(stream)
         if ev:
             ev[1].record(stream)
-        rc |= bsa.bsa_attn_prepare(plan, q, k, v, row_ptr, ws_attn, stream)
+        rc |= c.prepare(stream)
         if ev:
             ev[2].record(stream)
-        rc |= bsa.bsa_attn_run(plan, row_ptr, col_idx, o, ws_attn, stream)
+        rc |= c.run(stream)
         if ev:
             ev[3].record(stream)
         if rc:
@@ -169,9 +296,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if bsa.bsa_last_device_error(plan) != 0:
         raise RuntimeError("device error during warm-up")
-    flops = attention_flops(row_ptr.cpu().numpy(), col_idx.cpu().numpy(), w)
-    nnz_v = int(nnz.item())
-    rbytes = route_bytes(w, nnz_v, q.numel() * 2)
+    flops = c.flops()
+    rbytes = c.route_bytes()
+    density = c.density()               # kept fraction of the block mask
+    balance = c.balance()
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
@@ -194,39 +322,27 @@ def run_ours(args, rank, world, local_rank):
     total_ms = sum(step_ms)
 
     # the FP8 P.V variant on the same inputs and mask (reported beside the bf16 headline)
-    fp8_steps = max(3, min(args.steps, 50))
-    fp8_prep, fp8_run = [], []
-    for i in range(fp8_steps + 2):
-        flush.zero_()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        ev[0].record(stream)
-        rc = bsa.bsa_attn_prepare_fp8v(plan, q, k, v, row_ptr, ws_attn, stream)
-        ev[1].record(stream)
-        rc |= bsa.bsa_attn_run_fp8v(plan, row_ptr, col_idx, o, ws_attn, stream)
-        ev[2].record(stream)
-        if rc:
-            raise RuntimeError(f"fp8 attention call failed: {rc}")
-        if i >= 2:
-            fp8_prep.append(ev)
-    torch.cuda.synchronize()
+    fp8_steps = max(3, min(args.steps, 20))
+    fp8_prep_ms = timed_calls(torch, stream, flush, lambda s: bsa.bsa_attn_prepare_fp8v(
+        plan, c.q, c.k, c.v, c.row_ptr, c.ws_attn, s), fp8_steps)
+    fp8_run_ms = timed_calls(torch, stream, flush, lambda s: bsa.bsa_attn_run_fp8v(
+        plan, c.row_ptr, c.col_idx, c.o, c.ws_attn, s), fp8_steps)
     if bsa.bsa_last_device_error(plan) != 0:
         raise RuntimeError("device error in the fp8 variant")
-    fp8_prep_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in fp8_prep)
-    fp8_run_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in fp8_prep)
 
     # end to end through the public API with pinned host buffers
-    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (c.q, c.k, c.v))
+    oh = torch.empty(c.o.shape, dtype=c.o.dtype).pin_memory()
+    qd, kd, vd = torch.empty_like(c.q), torch.empty_like(c.k), torch.empty_like(c.v)
     e2e_steps = max(3, min(args.steps, 20))
 
     def e2e_step():
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        rp, ci, lh, nz = bsa.route(plan, qd, kd, p, w.k_floor, workspace=ws_route, col_cap=col_cap)
-        bsa.sparse_attn(plan, qd, kd, vd, rp, ci, workspace=ws_attn, out=o)
-        oh.copy_(o, non_blocking=True)
+        rp, ci, lh, nz = bsa.route(plan, qd, kd, p, w.k_floor, workspace=c.ws_route, col_cap=c.col_cap)
+        bsa.sparse_attn(plan, qd, kd, vd, rp, ci, workspace=c.ws_attn, out=c.o)
+        oh.copy_(c.o, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -239,19 +355,32 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    del qh, kh, vh, oh, qd, kd, vd
 
     (total_ms_max, e2e_ms_max, _, _), flops_sum = reduce_over_ranks(
         [total_ms, e2e_ms, max(attn_ms), max(route_ms)], flops, world, dev)
+    pk, pk_kind = peaks()
+    extras = {}
+    if not args.no_extras and rank == 0:
+        x_host = c.x
+        del c
+        torch.cuda.empty_cache()
+        for cid, pi in EXTRAS:
+            if cid == args.config:
+                continue
+            extras[f"config{cid}"] = extra_case(bsa, torch, dev, stream, flush, cid, pi, max(3, min(args.steps, 10)), pk)
+            torch.cuda.empty_cache()
+    else:
+        x_host = c.x
     if rank != 0:
         return None
 
-    pk, pk_kind = peaks()
     attn_avg = statistics.mean(attn_ms)
     achieved = flops / (attn_avg * 1e-3) / 1e12
-    traffic = load_traffic()
     ms_per_step = total_ms_max / args.steps
     value = flops_sum / (ms_per_step * 1e-3) / 1e12
     route_avg = statistics.mean(route_ms)
+    traffic = ATTN_TRAFFIC.get(sources_sha256(ATTN_SOURCES))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -264,29 +393,30 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) + sinusoidal (t,y,x) features, Wan2.1-480p-shaped; no weights)",
-        "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.N,
+        "data": "synthetic (seeded N(0,1) + sinusoidal (t,y,x) features, Wan-shaped video latents; no weights)",
+        "config": {"workload": workload_desc(w, args.p_index), "global_batch": w.B * world, "seq_len": w.N,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed before every timed step (256 MB write, untimed)",
-                   "density": round(float(nnz_v) / (w.rows * w.nb), 4)},
+                   "l2": "flushed before every timed call (256 MB write, untimed)",
+                   "density": round(density, 4)},
         "attn_ms_per_call": round(attn_avg, 4),
         "attn_tflops": round(achieved, 2),
         "attn_frac_of_bf16_burst": round(achieved / pk["bf16_tflops"], 4),
+        "attn_schedule": {"name": SCHEDULES[0][0], **balance},
         "route_ms_per_call": round(route_avg, 4),
         "route_gbs": round(rbytes / (route_avg * 1e-3) / 1e9, 1),
         "route_frac_of_hbm": round(rbytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "prepare_ms_per_call": round(statistics.mean(prep_ms), 4),
-        # the attention kernel is timed inside a ~1 s loop of steps under the power cap:
-        # the sustained bf16 peak is its denominator (the burst one is reported beside it)
+        # the attention kernel is timed per launch with CUDA events (each launch tens of
+        # ms, L2 flushed between launches): its denominator is the measured burst peak
         "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": round(achieved, 2),
-                     "peak": pk["bf16_tflops_sustained"],
-                     "peak_kind": f"bf16 dense sustained (cuBLAS 8192^3 for 4 s), {pk_kind}", "unit": "TFLOP/s",
-                     "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
-                     "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
+                     "peak": pk["bf16_tflops"],
+                     "peak_kind": f"bf16 dense burst (cuBLAS 8192^3, best of 10), {pk_kind}", "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops"], 4),
+                     "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
                      "traffic": traffic},
         "e2e": {"value": round(flops_sum / (e2e_ms_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms_max, 3),
-                "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2},
+                "h2d_bytes_per_step": 3 * w.B * w.N * w.H * w.d * 2, "d2h_bytes_per_step": w.B * w.N * w.H * w.d * 2},
         "attn_fp8v": {"kernel": ATTN_KERNEL + "<F8>", "calls": fp8_steps, "attn_ms_per_call": round(fp8_run_ms, 4),
                       "tflops": round(flops / (fp8_run_ms * 1e-3) / 1e12, 2),
                       "prepare_ms_per_call": round(fp8_prep_ms, 4),
@@ -294,40 +424,11 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
     }
+    if extras:
+        line["extra"] = extras
     if world == 1:
-        line["cpu_baseline"] = cpu_baseline(x, w, p, flops)
+        line["cpu_baseline"] = cpu_baseline(x_host, w, p, flops)
     return line
-
-
-ATTN_KERNEL = "k_attn_pp"        # the attention kernel bsa_attn_run launches for block 128
-ATTN_SOURCES = ("attn_pp.cu", "tc_common.cuh")
-ATTN_PROFILE = "k_attn_pp_wan21_480p.md"
-
-
-def sources_sha256(names):
-    import hashlib
-    h = hashlib.sha256()
-    for n in names:
-        h.update(open(os.path.join(ROOT, "block_sparse_attention_top_b200", "csrc", n), "rb").read())
-    return h.hexdigest()
-
-
-def load_traffic():
-    """DRAM bytes per launch of the attention kernel, from the committed ncu summary
-    (profiles/k_attn_pp_wan21_480p.md), or None if that summary was taken on
-    different kernel sources than the ones built here."""
-    path = os.path.join(ROOT, "profiles", ATTN_PROFILE)
-    try:
-        fields = {}
-        for line in open(path):
-            if ":" in line and line.startswith("- "):
-                key, val = line[2:].split(":", 1)
-                fields[key.strip()] = val.strip().strip("`")
-        if fields.get("sources sha256") != sources_sha256(ATTN_SOURCES):
-            return None
-        return int(fields["dram bytes per launch"].replace(",", ""))
-    except Exception:
-        return None
 
 
 # --------------------------------------------------------------------------- oracle (CPU)
@@ -393,12 +494,13 @@ def reference_step(x, w, p, full_flops, rng):
 
 def run_reference(args, world=1):
     """The fp64 CPU oracle on bounded samples of the same workload (the reference arm)."""
-    w = syn.workload(CID)
-    p = w.ps[P_INDEX]
-    x = syn.make_inputs(w, seed=syn.seed_for(CID, P_INDEX))
+    w = syn.workload(args.config)
+    p = w.ps[args.p_index]
+    x = syn.make_inputs(w, seed=syn.seed_for(args.config, args.p_index))
     import oracle
     r = oracle.route(x["q"], x["k"], w.T, w.Hs, w.Ws, w.block, p, w.k_floor)
     full_flops = attention_flops(r.row_ptr, r.col_idx, w)
+    density = float(r.row_ptr[-1]) / (w.rows * w.nb)
     rng = np.random.default_rng(1)
     for _ in range(args.warmup):
         reference_step(x, w, p, full_flops, rng)
@@ -410,8 +512,10 @@ def run_reference(args, world=1):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(w), "global_batch": w.B, "seq_len": w.N,
-                       "parallelism": "CPU oracle (numpy fp64)"},
+            "config": {"workload": workload_desc(w, args.p_index), "global_batch": w.B * world, "seq_len": w.N,
+                       "parallelism": "CPU oracle (numpy fp64)", "l2": "not applicable (host)",
+                       "density": round(density, 4)},
+            "ms_per_step_kind": "extrapolated from the timed per-step sample to the full step",
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -423,9 +527,17 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=CID, choices=[2, 3, 4],
+                    help="headline workload (routed configs; default 3: 720p)")
+    ap.add_argument("--p-index", type=int, default=None,
+                    help="index into the workload's Top-p values (default: p = 0.9 where listed)")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other full-size workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.p_index is None:
+        ps = syn.workload(args.config).ps
+        args.p_index = ps.index(0.9) if 0.9 in ps else 0
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

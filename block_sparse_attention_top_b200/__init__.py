@@ -40,6 +40,7 @@ BSA_OK, BSA_EINVAL, BSA_EUNSUPPORTED, BSA_ECAPACITY, BSA_EWORKSPACE, BSA_ECUDA, 
 BSA_ORDER_HILBERT2D_FRAME, BSA_ORDER_IDENTITY = 0, 1
 BSA_BF16, BSA_F32 = 0, 1
 BSA_OP_ROUTE, BSA_OP_ATTN, BSA_OP_MASK, BSA_OP_AUGMENT = 0, 1, 2, 3
+BSA_SCHED_L2_HEADS, BSA_SCHED_HEAVIEST_FIRST, BSA_SCHED_IN_ORDER = 0, 1, 2
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -50,6 +51,10 @@ _SIGS = {
     "bsa_plan_create": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _I]),
     "bsa_plan_destroy": (None, [_P]),
     "bsa_plan_info": (_I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
+    "bsa_plan_set_schedule": (_I, [_P, _I]),
+    "bsa_schedule_balance": (_I, [_P, _P, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64),
+                                  ctypes.POINTER(ctypes.c_double)]),
+    "bsa_attn_intermediates": (_I, [_P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P)]),
     "bsa_token_order": (_I, [_I, _I, _I, _I, _P]),
     "bsa_workspace_size": (_SZ, [_P, _I]),
     "bsa_route": (_I, [_P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
@@ -60,6 +65,7 @@ _SIGS = {
     "bsa_augment": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
     "bsa_sasa_budget": (_I, [_I, _P, ctypes.c_float, ctypes.c_float, ctypes.c_float, _P, _P, _P, _P, _P]),
     "bsa_rlb_plan": (_I, [_I, _I, _P, _P, _P, ctypes.POINTER(_I), _P, _P, _P]),
+    "bsa_rank_loads": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "bsa_rlb_gain": (_I, [_I, _P, _P, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                           _P, _P]),
     "bsa_mask_stripes": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I64, _P]),
@@ -123,6 +129,9 @@ class Plan:
         _check(_lib.bsa_plan_info(h, ctypes.byref(n), ctypes.byref(nb), ctypes.byref(rows)), "bsa_plan_info")
         self.N, self.nb, self.rows = n.value, nb.value, rows.value
 
+    def set_schedule(self, schedule: int) -> None:
+        _check(_lib.bsa_plan_set_schedule(self.handle, int(schedule)), "bsa_plan_set_schedule")
+
     def workspace_size(self, op: int) -> int:
         return int(_lib.bsa_workspace_size(self.handle, op))
 
@@ -139,6 +148,26 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def bsa_schedule_balance(plan, row_ptr, work):
+    """Per-CTA load balance of a work list (host tensors or arrays): (rho, max blocks, mean blocks)."""
+    rp = torch.as_tensor(row_ptr, dtype=torch.int32).cpu().contiguous()
+    wk = torch.as_tensor(work, dtype=torch.int32).cpu().contiguous()
+    if rp.numel() != plan.rows + 1 or wk.numel() != plan.rows:
+        raise ValueError("row_ptr must hold rows + 1 entries and work rows entries")
+    rho, mx, mean = ctypes.c_double(), _I64(), ctypes.c_double()
+    _check(_lib.bsa_schedule_balance(plan.handle, rp.data_ptr(), wk.data_ptr(), ctypes.byref(rho), ctypes.byref(mx),
+                                     ctypes.byref(mean)), "bsa_schedule_balance")
+    return rho.value, mx.value, mean.value
+
+
+def bsa_attn_intermediates(plan, workspace):
+    """Device addresses of (work list, e4m3 V tiles, V scales) in a prepared attention workspace."""
+    a, b, c = _P(), _P(), _P()
+    _check(_lib.bsa_attn_intermediates(plan.handle, _ptr(workspace), ctypes.byref(a), ctypes.byref(b),
+                                       ctypes.byref(c)), "bsa_attn_intermediates")
+    return a.value, b.value, c.value
 
 
 def bsa_token_order(T: int, Hs: int, Ws: int, order: int = BSA_ORDER_HILBERT2D_FRAME):
@@ -210,6 +239,21 @@ def bsa_rlb_plan(L_h, head_rank, R):
                              Ln.data_ptr(), rb.data_ptr(), ra.data_ptr()), "bsa_rlb_plan")
     mv = moves[:3 * n.value].view(-1, 3).tolist()
     return [tuple(m) for m in mv], Ln, float(rb[0]), float(ra[0])
+
+
+def bsa_rank_loads(L_h, head_rank, R):
+    """Host-only per-rank loads (Eq. 1), imbalance factor rho (Eq. 2) and head counts of a placement:
+    returns (L_r float32 [R], rho, heads_per_rank int32 [R])."""
+    Lh = torch.tensor([float(v) for v in L_h], dtype=torch.float32)
+    hr = torch.tensor([int(v) for v in head_rank], dtype=torch.int32)
+    if Lh.shape != hr.shape:
+        raise ValueError("L_h and head_rank must have the same length")
+    L_r = torch.empty(R, dtype=torch.float32)
+    cnt = torch.empty(R, dtype=torch.int32)
+    rho = ctypes.c_float()
+    _check(_lib.bsa_rank_loads(int(R), Lh.numel(), hr.data_ptr(), Lh.data_ptr(), L_r.data_ptr(), ctypes.byref(rho),
+                               cnt.data_ptr()), "bsa_rank_loads")
+    return L_r, rho.value, cnt
 
 
 def bsa_rlb_gain(L_r, L_r_new, c, P=0.0, C=0.0, A=0.0):
@@ -294,14 +338,17 @@ def balance_step(L_h_local, local_heads, tensors, rank, world, group=None, k1=1.
     for r, (hs, ls) in enumerate(every):
         for h, l in zip(hs, ls):
             owner[h], L_h[h] = r, l
-    L_r = [sum(ls) for _, ls in every]
-    rho = max(L_r) / (sum(L_r) / world) if sum(L_r) > 0 else 1.0
+    L_r, rho, _ = bsa_rank_loads(L_h, owner, world)
+    L_r = L_r.tolist()
     policy = bsa_balance_policy(rho, k1, k2)
     moves, L_r_new, rho_after = [], list(L_r), rho
     heads = list(local_heads)
+    new_owner = list(owner)
     if policy == 2:
         moves, L_new, _, rho_after = bsa_rlb_plan(L_h, owner, world)
         L_r_new = L_new.tolist()
+        for src, dst, h in moves:
+            new_owner[h] = dst
         out = []
         for x in tensors:
             x_new, heads_new = migrate_heads(x, list(local_heads), moves, rank, group)
@@ -314,7 +361,11 @@ def balance_step(L_h_local, local_heads, tensors, rank, world, group=None, k1=1.
             heads += [m[2] for m in moves if m[1] == rank]
     extra = [0] * len(heads)
     if policy >= 1:
-        counts = [len(hs) for hs, _ in every]
+        # heads each rank holds after the migration, in the order bsa_sasa_budget lists them
+        _, _, counts = bsa_rank_loads(L_h, new_owner, world)
+        counts = counts.tolist()
+        if counts[rank] != len(heads):
+            raise RuntimeError("head bookkeeping disagrees with the plan")
         _, _, _, ex = bsa_sasa_budget(L_r_new, n1, n2, heads_per_rank=counts)
         lo = sum(counts[:rank])
         extra = ex[lo:lo + counts[rank]].tolist()

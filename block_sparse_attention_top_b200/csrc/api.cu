@@ -72,10 +72,11 @@ AttnWs attn_ws_layout(const bsa_plan& p) {
     w.kp = off; off += align_up(tile);
     w.vp = off; off += align_up(tile);
     w.work = off; off += align_up((size_t)p.rows * sizeof(int32_t));
-    w.hist = off; off += align_up((size_t)(p.nb + 2) * sizeof(int32_t));
-    w.bins = off; off += align_up((size_t)(p.nb + 2) * sizeof(int32_t));
+    w.hist = off; off += align_up((size_t)sched_bins(p) * sizeof(int32_t));
+    w.bins = off; off += align_up((size_t)sched_bins(p) * sizeof(int32_t));
     w.counter = off; off += align_up(4 * sizeof(int32_t));
     w.vscale = off; off += align_up((size_t)p.B * p.H * p.d * sizeof(float));   // e4m3 V: per-channel scales
+    w.grank = off; off += align_up((size_t)p.B * p.H * sizeof(int32_t));       // head-group ranks
     w.total = off;
     return w;
 }
@@ -122,6 +123,8 @@ int bsa_plan_create(bsa_plan** out, int B, int H, int T, int Hs, int Ws,
     // element indices of [B,N,H,d] and of the padded tiles must fit in int64 and
     // row indices in int32
     if (N > (1ll << 30) || (int64_t)B * H * nb > (1ll << 30)) return BSA_EUNSUPPORTED;
+    // the attention kernels address the padded tiles with 32-bit row coordinates
+    if ((int64_t)B * H * nb * block > INT32_MAX) return BSA_EUNSUPPORTED;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ECUDA;
@@ -134,6 +137,7 @@ int bsa_plan_create(bsa_plan** out, int B, int H, int T, int Hs, int Ws,
     p->B = B; p->H = H; p->T = T; p->Hs = Hs; p->Ws = Ws; p->d = head_dim; p->block = block;
     p->order = order; p->N = N; p->nb = nb; p->rows = (int64_t)B * H * nb;
     p->device = dev; p->num_sms = prop.multiProcessorCount;
+    p->l2_bytes = prop.l2CacheSize; p->schedule = BSA_SCHED_L2_HEADS;
     std::vector<int32_t> perm((size_t)N);
     token_order(T, Hs, Ws, order, perm.data());
     if (cudaMalloc(&p->d_perm, (size_t)N * sizeof(int32_t)) != cudaSuccess ||
@@ -163,6 +167,50 @@ int bsa_plan_info(const bsa_plan* p, int64_t* N, int64_t* nb, int64_t* rows) {
     return BSA_OK;
 }
 
+int bsa_plan_set_schedule(bsa_plan* p, int schedule) {
+    if (!p) return BSA_EINVAL;
+    if (schedule != BSA_SCHED_L2_HEADS && schedule != BSA_SCHED_HEAVIEST_FIRST && schedule != BSA_SCHED_IN_ORDER)
+        return BSA_EINVAL;
+    p->schedule = schedule;
+    return BSA_OK;
+}
+
+int bsa_schedule_balance(const bsa_plan* p, const int32_t* row_ptr, const int32_t* work, double* rho,
+                         int64_t* max_blocks, double* mean_blocks) {
+    if (!p || !row_ptr || !work || !rho) return BSA_EINVAL;
+    // the attention kernels' static assignment: one CTA per SM, item k*grid + c
+    // to CTA c on even rounds k and to CTA grid - 1 - c on odd rounds
+    const int64_t grid = std::min<int64_t>(p->num_sms, p->rows);
+    std::vector<int64_t> load((size_t)grid, 0);
+    for (int64_t idx = 0; idx < p->rows; ++idx) {
+        const int64_t k = idx / grid, c = idx % grid;
+        const int64_t cta = (k & 1) ? grid - 1 - c : c;
+        const int32_t r = work[idx];
+        if (r < 0 || r >= p->rows) return BSA_EINVAL;
+        const int64_t n = (int64_t)row_ptr[r + 1] - row_ptr[r];
+        if (n < 0 || n > p->nb) return BSA_EINVAL;
+        load[(size_t)cta] += n;
+    }
+    int64_t mx = 0, sum = 0;
+    for (int64_t v : load) { mx = std::max(mx, v); sum += v; }
+    const double mean = grid > 0 ? (double)sum / (double)grid : 0.0;
+    *rho = mean > 0 ? (double)mx / mean : 1.0;
+    if (max_blocks) *max_blocks = mx;
+    if (mean_blocks) *mean_blocks = mean;
+    return BSA_OK;
+}
+
+int bsa_attn_intermediates(const bsa_plan* p, void* ws, const int32_t** work, const void** v_e4m3,
+                           const float** v_scale) {
+    if (!p || !ws) return BSA_EINVAL;
+    const AttnWs L = attn_ws_layout(*p);
+    char* base = (char*)ws;
+    if (work) *work = (const int32_t*)(base + L.work);
+    if (v_e4m3) *v_e4m3 = (const void*)(base + L.vp);
+    if (v_scale) *v_scale = (const float*)(base + L.vscale);
+    return BSA_OK;
+}
+
 size_t bsa_workspace_size(const bsa_plan* p, int op) {
     if (!p) return 0;
     if (op == BSA_OP_ROUTE) return route_ws_layout(*p).total;
@@ -189,6 +237,7 @@ int bsa_route(const bsa_plan* p, const void* q, const void* k, int dtype, float 
         (col_idx && misaligned(col_idx, 4)) || misaligned(L_h, 4) || misaligned(nnz, 8))
         return BSA_EINVAL;
     if (p->nb > kMaxRouteBlocks) return BSA_EUNSUPPORTED;
+    if (p->rows * p->nb > INT32_MAX) return BSA_EUNSUPPORTED;    // worst-case nnz must fit row_ptr (int32)
     const RouteWs L = route_ws_layout(*p);
     if (int rc = check_ws(ws, ws_bytes, L.total)) return rc;
     cudaStream_t s = (cudaStream_t)stream;
@@ -219,6 +268,7 @@ int bsa_augment(const bsa_plan* p, const int32_t* row_ptr, const uint16_t* order
     if (misaligned(row_ptr, 4) || misaligned(order, 2) || misaligned(extra, 4) || misaligned(row_ptr_out, 4) ||
         (col_idx_out && misaligned(col_idx_out, 4)) || misaligned(L_h_out, 4) || misaligned(nnz_out, 8))
         return BSA_EINVAL;
+    if (p->rows * p->nb > INT32_MAX) return BSA_EUNSUPPORTED;    // worst-case nnz must fit row_ptr (int32)
     if (int rc = check_ws(ws, ws_bytes, mask_ws_bytes(*p))) return rc;
     BSA_LAUNCH(launch_augment(*p, row_ptr, order, extra, (int32_t*)ws, row_ptr_out, col_idx_out, col_cap, L_h_out,
                               nnz_out, (cudaStream_t)stream));
@@ -257,6 +307,7 @@ int bsa_mask_window_anchor(const bsa_plan* p, int radius_frames, int n_anchor, i
         return BSA_EINVAL;
     if (col_cap < 0 || (col_cap > 0 && !col_idx)) return BSA_EINVAL;
     if (misaligned(row_ptr, 4) || (col_idx && misaligned(col_idx, 4)) || misaligned(nnz, 8)) return BSA_EINVAL;
+    if (p->rows * p->nb > INT32_MAX) return BSA_EUNSUPPORTED;    // worst-case nnz must fit row_ptr (int32)
     if (int rc = check_ws(ws, ws_bytes, mask_ws_bytes(*p))) return rc;
     BSA_LAUNCH(launch_mask_window_anchor(*p, radius_frames, n_anchor, step, (int32_t*)ws, row_ptr, col_idx, col_cap,
                                          nnz, (cudaStream_t)stream));
@@ -284,7 +335,7 @@ int bsa_attn_prepare(const bsa_plan* p, const void* q, const void* k, const void
     cudaStream_t s = (cudaStream_t)stream;
     char* base = (char*)ws;
     BSA_LAUNCH(launch_worklist(*p, row_ptr, (int32_t*)(base + L.hist), (int32_t*)(base + L.bins),
-                               (int32_t*)(base + L.work), s));
+                               (int32_t*)(base + L.grank), (int32_t*)(base + L.work), s));
     BSA_LAUNCH(launch_permute(*p, q, k, v, base + L.qp, base + L.kp, base + L.vp, s));
     return BSA_OK;
 }
@@ -340,7 +391,7 @@ int bsa_attn_prepare_fp8v(const bsa_plan* p, const void* q, const void* k, const
     cudaStream_t s = (cudaStream_t)stream;
     char* base = (char*)ws;
     BSA_LAUNCH(launch_worklist(*p, row_ptr, (int32_t*)(base + L.hist), (int32_t*)(base + L.bins),
-                               (int32_t*)(base + L.work), s));
+                               (int32_t*)(base + L.grank), (int32_t*)(base + L.work), s));
     BSA_LAUNCH(launch_permute(*p, q, k, v, base + L.qp, base + L.kp, nullptr, s, 2));
     BSA_LAUNCH(launch_quant_v(*p, v, (float*)(base + L.vscale), base + L.vp, s));
     return BSA_OK;

@@ -142,6 +142,28 @@ int bsa_rlb_plan(int R, int n_heads, const int32_t* head_rank, const float* L_h,
     return BSA_OK;
 }
 
+int bsa_rank_loads(int R, int n_heads, const int32_t* head_rank, const float* L_h, float* L_r, float* rho,
+                   int32_t* heads_per_rank) {
+    if (R < 1 || n_heads < 0 || (n_heads > 0 && (!head_rank || !L_h)) || !L_r) return BSA_EINVAL;
+    std::vector<double> L(R, 0.0);
+    std::vector<int32_t> cnt(R, 0);
+    for (int h = 0; h < n_heads; ++h) {
+        const int r = head_rank[h];
+        if (r < 0 || r >= R || !(L_h[h] >= 0.0f)) return BSA_EINVAL;
+        L[r] += L_h[h];                           // Eq. 1: a rank's load is the sum of its heads' loads
+        ++cnt[r];
+    }
+    double s = 0.0, m = 0.0;
+    for (int r = 0; r < R; ++r) {
+        L_r[r] = (float)L[r];
+        s += L[r];
+        m = std::max(m, L[r]);
+        if (heads_per_rank) heads_per_rank[r] = cnt[r];
+    }
+    if (rho) *rho = s > 0 ? (float)(m / (s / R)) : 1.0f;   // Eq. 2
+    return BSA_OK;
+}
+
 int bsa_rlb_gain(int R, const float* L_r, const float* L_r_new, double c, double P, double C, double A,
                  double* K, double* G) {
     if (R < 1 || !L_r || !L_r_new || !K || !G) return BSA_EINVAL;

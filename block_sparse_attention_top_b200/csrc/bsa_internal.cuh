@@ -12,6 +12,8 @@ struct bsa_plan {
     int64_t N, nb, rows;
     int device;
     int num_sms;
+    int64_t l2_bytes;    // the device's L2 size (sizes the head groups of BSA_SCHED_L2_HEADS)
+    int schedule;        // BSA_SCHED_*: order of the attention work list
     int32_t* d_perm;     // [N] raster index at reordered position
     int32_t* d_err;      // [4]: status, detail, spare, spare
 };
@@ -34,7 +36,7 @@ RouteWs route_ws_layout(const bsa_plan& p);
 inline size_t mask_ws_bytes(const bsa_plan& p) { return align_up((size_t)p.rows * sizeof(int32_t)); }
 
 struct AttnWs {
-    size_t qp, kp, vp, work, hist, bins, counter, vscale, total;
+    size_t qp, kp, vp, work, hist, bins, counter, vscale, grank, total;
 };
 AttnWs attn_ws_layout(const bsa_plan& p);
 
@@ -66,8 +68,13 @@ cudaError_t launch_augment(const bsa_plan& p, const int32_t* row_ptr, const uint
                            int32_t* counts, int32_t* row_ptr_out, int32_t* col_idx_out, int64_t col_cap,
                            float* L_h_out, int64_t* nnz_out, cudaStream_t s);
 
+// Work list in the plan's schedule.  hist and bins hold sched_bins(p) ints,
+// grank B*H ints.
+constexpr int kMaxSchedGroups = 8192;     // above: one group (heaviest-first)
+int sched_heads_per_group(const bsa_plan& p);
+int64_t sched_bins(const bsa_plan& p);
 cudaError_t launch_worklist(const bsa_plan& p, const int32_t* row_ptr, int32_t* hist,
-                            int32_t* bins, int32_t* work, cudaStream_t s);
+                            int32_t* bins, int32_t* grank, int32_t* work, cudaStream_t s);
 // n_tensors = 3: Q, K and V; 2: Q and K only (V goes through launch_quant_v)
 cudaError_t launch_permute(const bsa_plan& p, const void* q, const void* k, const void* v,
                            void* qp, void* kp, void* vp, cudaStream_t s, int n_tensors = 3);

@@ -1,12 +1,22 @@
-// Attention preparation: the heaviest-first work list and the reordered,
-// zero-padded Q/K/V tiles.
+// Attention preparation: the work list and the reordered, zero-padded Q/K/V
+// tiles.
 //
-// Work list: items (b, h, i) sorted by their number of key blocks, largest
-// first -- the single-GPU counterpart of the pages' runtime load balancing
-// (FVAttn review, section 3.2: the heavy heads set the critical path), which
-// here balances the persistent kernel's CTAs instead of ranks.  Counting sort
-// in three launches: histogram, descending bucket offsets, scatter.  The order
-// among items with the same count is unspecified (it does not change results).
+// Work list: the order in which the persistent attention kernel's CTAs take
+// the items (b, h, i) -- the single-GPU counterpart of the pages' runtime load
+// balancing (FVAttn review, section 3.2: the heavy heads set the critical
+// path), which here balances the kernel's CTAs instead of ranks.  Three
+// schedules (bsa_plan_set_schedule):
+//   BSA_SCHED_L2_HEADS        heads in groups whose K and V tiles fit a share
+//                             of L2, groups by descending total work, items of
+//                             a group by descending count: the CTAs that run
+//                             at the same time read the same few heads' tiles,
+//                             so those tiles are served from L2 (default);
+//   BSA_SCHED_HEAVIEST_FIRST  every item by descending count (longest
+//                             processing time first over all heads);
+//   BSA_SCHED_IN_ORDER        items in row order.
+// The sorted schedules are one counting sort on an ascending position key
+// (histogram, exclusive scan, scatter); the order among items with equal keys
+// is unspecified (it does not change results).
 //
 // Permutation: Xp[b, h, n', :] = X[b, perm[n'], h, :] for n' < N and zero for
 // the padding rows N <= n' < nb*block (FVAttn review, section 3.1: Hilbert
@@ -19,29 +29,59 @@
 namespace bsa {
 namespace {
 
-__global__ void k_hist(const int32_t* __restrict__ row_ptr, int64_t rows, int nb,
+// Rank of each head group by descending total work (ties: lower group first).
+// One CTA; a group is heads [g*G, (g+1)*G) and its rows are contiguous.
+__global__ void k_group_rank(const int32_t* __restrict__ row_ptr, int64_t rows, int64_t rows_per_group,
+                             int groups, int32_t* __restrict__ grank) {
+    extern __shared__ long long gw[];
+    for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+        const int64_t lo = (int64_t)g * rows_per_group, hi = min(rows, lo + rows_per_group);
+        gw[g] = (long long)row_ptr[hi] - (long long)row_ptr[lo];
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+        const long long wg = gw[g];
+        int rank = 0;
+        for (int u = 0; u < groups; ++u) rank += (gw[u] > wg || (gw[u] == wg && u < g)) ? 1 : 0;
+        grank[g] = rank;
+    }
+}
+
+// Position key of row r: bins are visited in ascending key order.
+struct SchedKey {
+    int nb;
+    int64_t rows_per_group;
+    const int32_t* grank;       // null: one group (plain heaviest-first)
+    __device__ int operator()(int64_t r, int n) const {
+        const int within = nb - n;                              // larger counts first
+        return grank ? grank[r / rows_per_group] * (nb + 1) + within : within;
+    }
+};
+
+__device__ __forceinline__ int row_count(const int32_t* row_ptr, int64_t r, int nb, int32_t* err) {
+    int n = row_ptr[r + 1] - row_ptr[r];
+    if (n < 0 || n > nb) {                       // malformed mask: record, clamp
+        if (err) record_error(err, BSA_EDEVICE, (int)r);
+        n = n < 0 ? 0 : nb;
+    }
+    return n;
+}
+
+__global__ void k_hist(const int32_t* __restrict__ row_ptr, int64_t rows, SchedKey key,
                        int32_t* __restrict__ hist, int32_t* err) {
     const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
-    int n = row_ptr[r + 1] - row_ptr[r];
-    if (n < 0 || n > nb) {                       // malformed mask: record, clamp
-        record_error(err, BSA_EDEVICE, (int)r);
-        n = n < 0 ? 0 : nb;
-    }
-    atomicAdd(&hist[n], 1);
+    atomicAdd(&hist[key(r, row_count(row_ptr, r, key.nb, err))], 1);
 }
 
-// bins[n] = number of items with a count greater than n (start of bucket n in
-// descending order).  One CTA; nb + 1 buckets.
-__global__ void k_bins(const int32_t* __restrict__ hist, int nb, int32_t* __restrict__ bins) {
+// bins[u] = number of items whose key is below u (exclusive scan).  One CTA.
+__global__ void k_bins(const int32_t* __restrict__ hist, int n_bins, int32_t* __restrict__ bins) {
     __shared__ int wsum[32];
     const int tid = threadIdx.x;
-    const int buckets = nb + 1;
-    const int per = (buckets + blockDim.x - 1) / blockDim.x;
-    // walk buckets from the top: position u corresponds to bucket nb - u
-    const int lo = tid * per, hi = min(buckets, lo + per);
+    const int per = (n_bins + blockDim.x - 1) / blockDim.x;
+    const int lo = min(n_bins, tid * per), hi = min(n_bins, lo + per);
     int run = 0;
-    for (int u = lo; u < hi; ++u) run += hist[nb - u];
+    for (int u = lo; u < hi; ++u) run += hist[u];
     int incl = run;
     const int lane = tid % 32, wid = tid / 32;
     for (int o = 1; o < 32; o <<= 1) {
@@ -53,19 +93,26 @@ __global__ void k_bins(const int32_t* __restrict__ hist, int nb, int32_t* __rest
     int off = incl - run;
     for (int w = 0; w < wid; ++w) off += wsum[w];
     for (int u = lo; u < hi; ++u) {
-        bins[nb - u] = off;
-        off += hist[nb - u];
+        bins[u] = off;
+        off += hist[u];
     }
 }
 
-__global__ void k_scatter(const int32_t* __restrict__ row_ptr, int64_t rows, int nb,
+__global__ void k_scatter(const int32_t* __restrict__ row_ptr, int64_t rows, SchedKey key,
                           int32_t* __restrict__ bins, int32_t* __restrict__ work) {
     const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
-    int n = row_ptr[r + 1] - row_ptr[r];
-    n = n < 0 ? 0 : (n > nb ? nb : n);
-    const int pos = atomicAdd(&bins[n], 1);
+    const int pos = atomicAdd(&bins[key(r, row_count(row_ptr, r, key.nb, nullptr))], 1);
     work[pos] = (int32_t)r;
+}
+
+// In-order schedule: work[r] = r (the counts are still checked).
+__global__ void k_iota(const int32_t* __restrict__ row_ptr, int64_t rows, int nb, int32_t* __restrict__ work,
+                       int32_t* err) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    row_count(row_ptr, r, nb, err);
+    work[r] = (int32_t)r;
 }
 
 // One thread moves 16 bytes.  Destination rows are visited in (b, n', h)
@@ -92,15 +139,47 @@ __global__ void k_permute(const uint4* __restrict__ q, const uint4* __restrict__
 
 }  // namespace
 
+int sched_heads_per_group(const bsa_plan& p) {
+    // K and V tiles of one head: 2 * nb * block * d bf16 values
+    const double head_bytes = 2.0 * (double)p.nb * p.block * p.d * 2.0;
+    const double budget = 0.4 * (double)p.l2_bytes;
+    const int g = (int)(budget / head_bytes);
+    return g < 1 ? 1 : (g > p.B * p.H ? p.B * p.H : g);
+}
+
+int64_t sched_bins(const bsa_plan& p) {
+    const int64_t heads = (int64_t)p.B * p.H;
+    return (heads + 1) * (p.nb + 1);
+}
+
 cudaError_t launch_worklist(const bsa_plan& p, const int32_t* row_ptr, int32_t* hist, int32_t* bins,
-                            int32_t* work, cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)(p.nb + 1) * sizeof(int32_t), s);
-    if (e != cudaSuccess) return e;
+                            int32_t* grank, int32_t* work, cudaStream_t s) {
     const int t = 256;
     const unsigned g = (unsigned)((p.rows + t - 1) / t);
-    k_hist<<<g, t, 0, s>>>(row_ptr, p.rows, (int)p.nb, hist, p.d_err);
-    k_bins<<<1, 1024, 0, s>>>(hist, (int)p.nb, bins);
-    k_scatter<<<g, t, 0, s>>>(row_ptr, p.rows, (int)p.nb, bins, work);
+    if (p.schedule == BSA_SCHED_IN_ORDER) {
+        k_iota<<<g, t, 0, s>>>(row_ptr, p.rows, (int)p.nb, work, p.d_err);
+        return cudaGetLastError();
+    }
+    SchedKey key{(int)p.nb, p.rows, nullptr};
+    int n_bins = (int)p.nb + 1;
+    const int G = sched_heads_per_group(p);
+    const int groups = (int)((p.B * p.H + G - 1) / G);
+    if (p.schedule == BSA_SCHED_L2_HEADS && groups > 1 && groups <= kMaxSchedGroups) {
+        key.rows_per_group = (int64_t)G * p.nb;
+        key.grank = grank;
+        n_bins = groups * ((int)p.nb + 1);
+        const size_t smem = (size_t)groups * sizeof(long long);
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(k_group_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        k_group_rank<<<1, 1024, smem, s>>>(row_ptr, p.rows, key.rows_per_group, groups, grank);
+    }
+    cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)n_bins * sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+    k_hist<<<g, t, 0, s>>>(row_ptr, p.rows, key, hist, p.d_err);
+    k_bins<<<1, 1024, 0, s>>>(hist, n_bins, bins);
+    k_scatter<<<g, t, 0, s>>>(row_ptr, p.rows, key, bins, work);
     return cudaGetLastError();
 }
 

@@ -187,8 +187,8 @@ k_scores(const double* __restrict__ qbar, const double* __restrict__ kbar, doubl
 // Row routing, one warp per row (nb <= 1024).  Each lane holds E = nbp/32
 // consecutive elements of the padded row as one 64-bit key that sorts in
 // ascending order exactly as (s descending, j ascending): the order-preserving
-// image of s, complemented, with its 10 lowest bits replaced by j.  (Dropping
-// those bits only merges scores equal to ~1e-13 relative, far inside the 1e-6
+// image of s, complemented, with its 13 lowest bits replaced by j.  (Dropping
+// those bits only merges scores equal to ~1e-12 relative, far inside the 1e-6
 // tie tolerance, and then orders them by ascending j as the exact rule does.)
 // A bitonic network sorts the keys: exchanges between registers for strides
 // below E, between lanes (shuffles) above.  P, the inclusive cumulative mass

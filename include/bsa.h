@@ -73,6 +73,11 @@ extern "C" {
 #define BSA_OP_MASK  2
 #define BSA_OP_AUGMENT 3
 
+/* ---- attention work-list schedules (bsa_plan_set_schedule) ---- */
+#define BSA_SCHED_L2_HEADS       0   /* head groups sized to L2, heaviest group first, heaviest items first */
+#define BSA_SCHED_HEAVIEST_FIRST 1   /* every item by descending key-block count */
+#define BSA_SCHED_IN_ORDER       2   /* items in row order */
+
 typedef struct bsa_plan bsa_plan;
 
 /*
@@ -95,6 +100,37 @@ void bsa_plan_destroy(bsa_plan* plan);
 
 /* Host-only shape query: N tokens, nb blocks per head, rows = B*H*nb. */
 int bsa_plan_info(const bsa_plan* plan, int64_t* N, int64_t* nb, int64_t* rows);
+
+/*
+ * Host-only: choose the order in which the attention kernel's persistent CTAs
+ * take the work items (b, h, i); it changes the speed, never the result.  It
+ * is the single-GPU form of the FVAttn review's runtime load balancing
+ * (section 3 "Stage 2" and section 3.2: the heavy heads set the critical
+ * path): the balance is across the kernel's CTAs instead of across ranks.
+ *   BSA_SCHED_L2_HEADS (the default): heads are cut into groups whose K and V
+ *     tiles take at most 40 % of the device's L2; groups run in descending
+ *     total work and the items of a group in descending key-block count, so
+ *     the CTAs that run at the same time share the tiles of a few heads;
+ *   BSA_SCHED_HEAVIEST_FIRST: every item in descending count (over all heads);
+ *   BSA_SCHED_IN_ORDER: rows in index order.
+ * Takes effect at the next bsa_attn_prepare / bsa_attn_prepare_fp8v.
+ * BSA_EINVAL for an unknown schedule.
+ */
+int bsa_plan_set_schedule(bsa_plan* plan, int schedule);
+
+/*
+ * Host-only: the single-GPU analogue of the review's imbalance factor (Eq.
+ * 2, rho = max load / mean load) for one work list: the load of a CTA is
+ * the number of key blocks of the items the attention kernel assigns to it
+ * (one CTA per SM; item k*grid + c goes to CTA c on even rounds k and to
+ * CTA grid - 1 - c on odd rounds, grid = min(SM count, rows)).  row_ptr:
+ * the mask's row_ptr; work: the work list of a prepared attention workspace
+ * (bsa_attn_intermediates), both copied to HOST memory.  *rho, and the
+ * largest and mean CTA loads when not NULL.  BSA_EINVAL for null pointers or
+ * an invalid work list.
+ */
+int bsa_schedule_balance(const bsa_plan* plan, const int32_t* row_ptr, const int32_t* work, double* rho,
+                         int64_t* max_blocks, double* mean_blocks);
 
 /*
  * Host-only: write the token permutation of a (T, Hs, Ws) grid under `order`
@@ -219,11 +255,24 @@ int bsa_rlb_plan(int R, int n_heads, const int32_t* head_rank, const float* L_h,
                  int* n_moves, float* L_r_new, float* rho_before, float* rho_after);
 
 /*
+ * Host-only: per-rank workloads and the imbalance factor of a head placement
+ * (FVAttn review, section 3 "Stage 2", Eqs. 1-2): L_r[r] = sum of L_h[h] over
+ * the heads with head_rank[h] == r, *rho = max_r L_r / mean_r L_r (1 when
+ * every load is 0).  heads_per_rank (int32 [R], may be NULL) receives the
+ * number of heads each rank holds.  rho may be NULL.  BSA_EINVAL for R < 1,
+ * n_heads < 0, null arrays, a rank outside [0, R) or a negative workload.
+ * Host pointers; no CUDA call.
+ */
+int bsa_rank_loads(int R, int n_heads, const int32_t* head_rank, const float* L_h, float* L_r, float* rho,
+                   int32_t* heads_per_rank);
+
+/*
  * Host-only: the review's gain model for a migration plan (section 3 "Stage
  * 2", Eqs. 3-4, and the joint form of Eq. 11): the straggler time saved
  * K = c * (max_r L_r - max_r L_r_new), with c the time per unit of workload,
- * and the net gain G = K - P - C - A, with P the plan-search time, C the
- * communication time of the migration and A the slack-augmentation cost (0
+ * and the net gain G = K - P - C - A, with P the communication cost of
+ * moving the migrated heads' state, C the scheduling cost of solving the
+ * migration plan and A the slack-augmentation cost (0
  * without augmentation; the pages give no values for c, P, C or A).  L_r,
  * L_r_new: [R] host arrays (e.g. from bsa_rlb_plan).  Negative status for
  * R < 1, null pointers or negative loads.
@@ -297,8 +346,8 @@ int bsa_sparse_attn(const bsa_plan* plan, const void* q, const void* k, const vo
 
 /*
  * The two halves of bsa_sparse_attn, for callers that time or overlap them.
- * prepare: orders the work items (b,h,i) heaviest first by their number of
- *   key blocks, and copies Q, K, V into reordered, zero-padded
+ * prepare: orders the work items (b,h,i) in the plan's schedule
+ *   (bsa_plan_set_schedule), and copies Q, K, V into reordered, zero-padded
  *   [B, H, nb*block, d] bf16 tiles inside the workspace.
  * run: the persistent tcgen05 attention kernel over that work list (for
  *   block 128: two softmax warp groups on alternating key blocks, QK and PV
@@ -334,6 +383,16 @@ int bsa_attn_prepare_fp8v(const bsa_plan* plan, const void* q, const void* k, co
                           const int32_t* row_ptr, void* workspace, size_t ws_bytes, void* stream);
 int bsa_attn_run_fp8v(const bsa_plan* plan, const int32_t* row_ptr, const int32_t* col_idx,
                       void* o, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Host-only: device addresses of the pieces of a prepared attention
+ * workspace, for inspection: the work list (int32 [rows], row indices in
+ * the order the kernel takes them), the e4m3 V tiles of the FP8 variant
+ * (bytes [B*H*nb*d, 128]: per (head, key block) d rows of 128 keys) and
+ * their per-channel scales (float [B*H*d]).  Any output may be NULL.
+ */
+int bsa_attn_intermediates(const bsa_plan* plan, void* workspace, const int32_t** work, const void** v_e4m3,
+                           const float** v_scale);
 
 /*
  * Same contract as bsa_attn_run, computed by a slow CUDA-core kernel (one

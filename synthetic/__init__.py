@@ -1,10 +1,11 @@
 """Seeded synthetic inputs shaped like video-DiT self-attention activations.
 
 This module is shared by the CUDA path's tests/bench and by the oracle's tests.
-It holds no routing or attention arithmetic: only the random draws, the
-positional "feature" signal mixed into Q/K, the fp32 -> bf16 encoding of the
-drawn values, and the fixed window-plus-anchor block pattern used by the
-long-horizon workload (an *input* mask, never produced by routing).
+It holds no routing, masking or attention arithmetic: only the random draws,
+the positional "feature" signal mixed into Q/K and the fp32 -> bf16 encoding
+of the drawn values.  The long-horizon workload's fixed window-plus-anchor
+mask is not drawn here: tests take it from the oracle (oracle/masks.py) and
+the benchmark from the library's own device producer.
 
 Layout of every Q/K/V tensor: [B, N, H, d] in C order, N = T*Hs*Ws tokens in
 raster order (frame t, then row y, then column x), i.e. the layout a video DiT
@@ -37,7 +38,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "CONFIGS", "workload", "make_inputs", "features",
-    "f32_to_bf16_bits", "bf16_bits_to_f32", "window_anchor_mask",
+    "f32_to_bf16_bits", "bf16_bits_to_f32", "seed_for",
 ]
 
 
@@ -84,14 +85,24 @@ def workload(cid: int, **override) -> Workload:
     return dataclasses.replace(w, **override) if override else w
 
 
-def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+def f32_to_bf16_bits_reference(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (nearest, ties to even); returns the uint16 bit patterns.
 
-    Inputs here are finite, so no NaN handling is needed.
+    The definition written out on the bit patterns (add 0x7FFF plus the lowest
+    kept bit, drop the low 16 bits).  Inputs here are finite, so no NaN
+    handling is needed.
     """
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
     rounded = u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))
     return (rounded >> np.uint32(16)).astype(np.uint16)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """As f32_to_bf16_bits_reference (same bits, checked by the tests), through
+    torch's multi-threaded CPU conversion, which rounds the same way."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -161,33 +172,6 @@ def make_inputs(w: Workload | int, sub: int = 0, seed: int | None = None) -> dic
         out[name] = z if w.dtype == "f32" else f32_to_bf16_bits(z)
         del z
     return out
-
-
-def window_anchor_mask(w: Workload, step: int = 0, radius: int = 2, n_anchor: int = 8):
-    """Fixed block pattern: a local window of +-`radius` latent frames plus
-    `n_anchor` global anchor key blocks that move with the diffusion step.
-
-    The pattern is stated on block indices of the frame-major order (frames
-    stay contiguous there, so block i covers frames
-    [i*block // (Hs*Ws), ((i+1)*block - 1) // (Hs*Ws)]).  Key block j is kept
-    for query block i iff their frame ranges come within `radius` frames; the
-    anchors are A(step) = {(step + m*(nb // n_anchor)) mod nb, m < n_anchor},
-    the same for every row and head.  Returns (row_ptr int32 [B*H*nb+1],
-    col_idx int32 [nnz]) with columns ascending and unique, rows ordered
-    (b*H + h)*nb + i.
-    """
-    nb, hw = w.nb, w.Hs * w.Ws
-    first = np.arange(nb) * w.block // hw
-    last = (np.minimum((np.arange(nb) + 1) * w.block, w.N) - 1) // hw
-    near = (first[None, :] <= last[:, None] + radius) & (last[None, :] >= first[:, None] - radius)
-    anchors = (step + np.arange(n_anchor) * (nb // n_anchor)) % nb
-    near[:, anchors] = True
-    counts = near.sum(axis=1)
-    cols = np.nonzero(near)[1].astype(np.int32)
-    reps = w.B * w.H
-    row_ptr = np.zeros(reps * nb + 1, dtype=np.int64)
-    row_ptr[1:] = np.cumsum(np.tile(counts, reps))
-    return row_ptr.astype(np.int32), np.tile(cols, reps)
 
 
 def seed_for(cid: int, p_index: int = 0) -> int:

@@ -5,6 +5,7 @@ import pytest
 import torch
 
 import oracle
+import oracle.masks as om
 import synthetic as syn
 from _gpu import bf16_to_f64, to_dev
 from _parity import check_attention, sample_blocks
@@ -159,7 +160,7 @@ def test_malformed_mask_reported(bsa, kernel, block):
 
 
 @pytest.mark.parametrize("kernel", ["tc"])
-@pytest.mark.parametrize("cid,p_index", [(2, 0), (3, 1), (4, 0)])
+@pytest.mark.parametrize("cid,p_index", [(2, 0), (3, 0), (3, 1), (3, 2), (4, 0)])
 def test_full_size_routed_sampled(bsa, kernel, cid, p_index):
     w = syn.workload(cid)
     x = syn.make_inputs(w, seed=syn.seed_for(cid, p_index))
@@ -175,7 +176,7 @@ def test_full_size_routed_sampled(bsa, kernel, cid, p_index):
 def test_long_fixed_mask_sampled(bsa, kernel, step):
     w = syn.workload(5)
     x = syn.make_inputs(w, seed=syn.seed_for(5))
-    row_ptr, col_idx = syn.window_anchor_mask(w, step=step)
+    row_ptr, col_idx = om.window_anchor_csr(w.B, w.H, w.N, w.block, w.Hs * w.Ws, 2, 8, step)
     o, status = gpu_attn(bsa, w, x["q"], x["k"], x["v"], row_ptr, col_idx, kernel)
     assert status == 0
     counts = np.diff(row_ptr)

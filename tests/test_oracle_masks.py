@@ -37,12 +37,3 @@ def test_window_properties_on_long_shape():
             assert (j in cols) == (near or j in anchors)
             if near:
                 assert i in rows[j]                   # the window part is symmetric
-
-
-def test_matches_the_input_generators_pattern():
-    """The seeded workloads draw their config-5 mask with the same reading."""
-    w = syn.workload(5, T=9, Hs=6, Ws=10, H=2, block=32)
-    for step in (0, 1, 2):
-        rp, ci = syn.window_anchor_mask(w, step=step)
-        orp, oci = om.window_anchor_csr(w.B, w.H, w.N, w.block, w.Hs * w.Ws, 2, 8, step)
-        assert np.array_equal(rp, orp) and np.array_equal(ci, oci)

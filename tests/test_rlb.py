@@ -83,3 +83,27 @@ def test_gain_model_matches_oracle(bsa):
         assert bsa.bsa_rlb_gain(L, Ln, c, P, C, A=0.25)[1] == pytest.approx(Go - 0.25, abs=1e-12)
     with pytest.raises(bsa.BsaError):
         bsa.bsa_rlb_gain([1.0, -2.0], [1.0, 1.0], 1.0)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_rank_loads_match_oracle(bsa, seed):
+    """Eq. 1 per-rank loads, Eq. 2 rho and head counts of a random placement."""
+    rng = np.random.default_rng(100 + seed)
+    R = int(rng.integers(1, 9))
+    L_h, owner = _case(rng, R, hmin=0, hmax=4)
+    owner = list(rng.permutation(owner))
+    L_r, rho, cnt = bsa.bsa_rank_loads(L_h, owner, R)
+    want = orlb.rank_loads(L_h.astype(np.float64), owner, R)
+    np.testing.assert_allclose(L_r.numpy(), want, rtol=1e-6)
+    if want.sum() > 0:
+        assert rho == pytest.approx(orlb.rho(want), rel=1e-6)
+    assert cnt.tolist() == [owner.count(r) for r in range(R)]
+
+
+def test_rank_loads_errors(bsa):
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_rank_loads([1.0, 2.0], [0, 3], 2)          # rank outside [0, R)
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_rank_loads([1.0, -2.0], [0, 1], 2)         # negative workload
+    L_r, rho, cnt = bsa.bsa_rank_loads([0.0, 0.0], [0, 1], 2)
+    assert rho == 1.0 and cnt.tolist() == [1, 1]
