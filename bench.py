@@ -155,9 +155,9 @@ def sources_sha256(names):
 class Case:
     """One workload resident on the device: inputs, plan, mask buffers, workspaces."""
 
-    def __init__(self, bsa, torch, dev, cid, p_index, rank=0):
+    def __init__(self, bsa, torch, dev, cid, p_index, rank=0, heads=None):
         self.bsa, self.torch, self.dev = bsa, torch, dev
-        self.w = w = syn.workload(cid)
+        self.w = w = syn.workload(cid, H=heads) if heads else syn.workload(cid)
         self.p_index = p_index
         self.p = w.ps[p_index] if p_index is not None else None
         seed = syn.seed_for(cid, p_index or 0) + 7919 * rank
@@ -272,8 +272,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)     # > 126 MB L2
-    c = Case(bsa, torch, dev, args.config, args.p_index, rank)
+    c = Case(bsa, torch, dev, args.config, args.p_index, rank, heads=args.heads)
     w, p, plan = c.w, c.p, c.plan
+    plan.set_schedule(dict(SCHEDULES)[args.schedule])
 
     def step(ev=None):
         if ev:
@@ -320,6 +321,18 @@ def run_ours(args, rank, world, local_rank):
     prep_ms = [e[1].elapsed_time(e[2]) for e in events]
     attn_ms = [e[2].elapsed_time(e[3]) for e in events]
     total_ms = sum(step_ms)
+    if args.step_only:
+        # profiler captures: the timed step alone, nothing after it
+        return {"metric": METRIC, "value": round(flops / (total_ms / args.steps * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": workload_desc(w, args.p_index), "schedule": args.schedule,
+                           "density": round(density, 4), "step_only": True},
+                "attn_ms_per_call": round(statistics.mean(attn_ms), 4),
+                "attn_tflops": round(flops / (statistics.mean(attn_ms) * 1e-3) / 1e12, 2),
+                "route_ms_per_call": round(statistics.mean(route_ms), 4),
+                "attn_schedule": {"name": args.schedule, **balance}} if rank == 0 else None
 
     # the FP8 P.V variant on the same inputs and mask (reported beside the bf16 headline)
     fp8_steps = max(3, min(args.steps, 20))
@@ -401,7 +414,7 @@ def run_ours(args, rank, world, local_rank):
         "attn_ms_per_call": round(attn_avg, 4),
         "attn_tflops": round(achieved, 2),
         "attn_frac_of_bf16_burst": round(achieved / pk["bf16_tflops"], 4),
-        "attn_schedule": {"name": SCHEDULES[0][0], **balance},
+        "attn_schedule": {"name": args.schedule, **balance},
         "route_ms_per_call": round(route_avg, 4),
         "route_gbs": round(rbytes / (route_avg * 1e-3) / 1e9, 1),
         "route_frac_of_hbm": round(rbytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
@@ -532,6 +545,12 @@ def main():
     ap.add_argument("--p-index", type=int, default=None,
                     help="index into the workload's Top-p values (default: p = 0.9 where listed)")
     ap.add_argument("--no-extras", action="store_true", help="skip the other full-size workloads")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the headline workload's head count (smaller cases for profiler captures)")
+    ap.add_argument("--schedule", choices=[n for n, _ in SCHEDULES], default=SCHEDULES[0][0],
+                    help="work-list schedule of the headline workload")
+    ap.add_argument("--step-only", action="store_true",
+                    help="time the headline step only (no FP8 variant, end to end, extras or CPU baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

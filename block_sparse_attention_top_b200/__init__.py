@@ -52,6 +52,7 @@ _SIGS = {
     "bsa_plan_destroy": (None, [_P]),
     "bsa_plan_info": (_I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
     "bsa_plan_set_schedule": (_I, [_P, _I]),
+    "bsa_plan_set_wait_limit": (_I, [_P, ctypes.c_uint64]),
     "bsa_schedule_balance": (_I, [_P, _P, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64),
                                   ctypes.POINTER(ctypes.c_double)]),
     "bsa_attn_intermediates": (_I, [_P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P)]),
@@ -69,6 +70,7 @@ _SIGS = {
     "bsa_rlb_gain": (_I, [_I, _P, _P, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                           _P, _P]),
     "bsa_mask_stripes": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I64, _P]),
+    "bsa_mask_stripes_device": (_I, [_P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "bsa_balance_policy": (_I, [ctypes.c_float, ctypes.c_float, ctypes.c_float]),
     "bsa_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bsa_attn_prepare": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -131,6 +133,9 @@ class Plan:
 
     def set_schedule(self, schedule: int) -> None:
         _check(_lib.bsa_plan_set_schedule(self.handle, int(schedule)), "bsa_plan_set_schedule")
+
+    def set_wait_limit(self, ns: int) -> None:
+        _check(_lib.bsa_plan_set_wait_limit(self.handle, int(ns)), "bsa_plan_set_wait_limit")
 
     def workspace_size(self, op: int) -> int:
         return int(_lib.bsa_workspace_size(self.handle, op))
@@ -285,6 +290,17 @@ def bsa_mask_stripes(B, H, T, Hs, Ws, block, params, order=0):
     return row_ptr, col_idx[:nnz.value].clone()
 
 
+def bsa_mask_stripes_device(plan, params, row_ptr, col_idx, col_cap, nnz, workspace, stream=None):
+    """Device stripe-mask CSR into device row_ptr / col_idx / nnz; params: H rows of
+    (w_t, o_t, s_t, w_s, o_s, s_s) (host)."""
+    pr = torch.tensor([[int(v) for v in row] for row in params], dtype=torch.int32).reshape(-1)
+    if pr.numel() != 6 * plan.H:
+        raise ValueError("params must hold 6 values per head")
+    return _lib.bsa_mask_stripes_device(plan.handle, pr.data_ptr(), _ptr(row_ptr), _ptr(col_idx), int(col_cap),
+                                        _ptr(nnz), _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                        _stream(stream))
+
+
 def bsa_balance_policy(rho, k1=1.05, k2=1.10) -> int:
     return _lib.bsa_balance_policy(float(rho), float(k1), float(k2))
 
@@ -371,6 +387,75 @@ def balance_step(L_h_local, local_heads, tensors, rank, world, group=None, k1=1.
         extra = ex[lo:lo + counts[rank]].tolist()
     return dict(policy=policy, rho_before=rho, rho_after=rho_after, moves=moves, L_r=L_r, L_r_new=L_r_new,
                 tensors=tensors, local_heads=heads, extra=extra)
+
+
+def return_heads(out, heads, home_heads, moves, rank, group=None):
+    """The reverse of migrate_heads: send every migrated head's output back to the rank it came from
+    and return this rank's outputs in its original head order (FVAttn review, section 3 "Block-Sparse
+    Attention Execution": the outputs of migrated heads go back and head order is restored).
+
+    out: [B, N, H_now, d] outputs of the heads listed in `heads` (the order balance_step / migrate_heads
+    returned); home_heads: this rank's heads before the migration, in their original order; moves: the
+    plan's [(src, dst, head)].  Returns [B, N, len(home_heads), d].  Plumbing only."""
+    import torch.distributed as dist
+    home_of = {h: src for src, dst, h in moves}            # heads that moved: where they live
+    reqs, kept, got = [], {}, {}
+    for i, h in enumerate(heads):
+        if h in home_of and home_of[h] != rank:            # computed here for another rank: send it home
+            reqs.append(dist.isend(out[:, :, i].contiguous(), home_of[h], group=group))
+        else:
+            kept[h] = out[:, :, i]
+    for src, dst, h in moves:
+        if src == rank:                                    # ours, computed elsewhere: receive it
+            buf = torch.empty_like(out[:, :, 0]) if out.shape[2] else torch.empty(
+                out.shape[:2] + out.shape[3:], dtype=out.dtype, device=out.device)
+            reqs.append(dist.irecv(buf, dst, group=group))
+            got[h] = buf
+    for q in reqs:
+        q.wait()
+    parts = []
+    for h in home_heads:
+        if h in kept:
+            parts.append(kept[h])
+        elif h in got:
+            parts.append(got[h])
+        else:
+            raise RuntimeError(f"head {h} is neither kept nor received on rank {rank}")
+    return torch.stack(parts, dim=2) if parts else out[:, :, :0]
+
+
+def local_attention(q, k, v, T, Hs, Ws, block, p, k_floor, extra=None):
+    """Route and attend over the heads a rank holds: bf16 [B, N, H_local, d] on its device; extra: SASA
+    blocks per local head (bsa_augment), or None.  Returns (o, L_h) device tensors."""
+    B, N, H, d = q.shape
+    plan = Plan(B, H, T, Hs, Ws, d, block)
+    ws = plan.workspace(BSA_OP_ROUTE, q.device)
+    row_ptr, col_idx, L_h, _ = route(plan, q, k, p, k_floor, workspace=ws)
+    if extra is not None and any(int(e) > 0 for e in extra):
+        ex = torch.tensor([int(e) for e in extra], dtype=torch.int32, device=q.device)
+        rp2 = torch.empty_like(row_ptr)
+        ci2 = torch.empty(plan.rows * plan.nb, dtype=torch.int32, device=q.device)
+        L2 = torch.empty_like(L_h)
+        nnz2 = torch.empty(1, dtype=torch.int64, device=q.device)
+        ws_aug = plan.workspace(BSA_OP_AUGMENT, q.device)
+        _check(bsa_augment(plan, row_ptr, bsa_route_order(plan, ws), ex, rp2, ci2, ci2.numel(), L2, nnz2, ws_aug),
+               "bsa_augment")
+        row_ptr, col_idx, L_h = rp2, ci2, L2
+    o = sparse_attn(plan, q, k, v, row_ptr, col_idx)
+    _check(bsa_last_device_error(plan), "device error")
+    return o, L_h
+
+
+def balanced_attention(q, k, v, L_h_local, local_heads, rank, world, compute, group=None, **policy):
+    """One balanced attention step over the ranks (FVAttn review, section 3): balance_step moves the
+    planned heads' Q, K, V and decides the augmentation, `compute(q, k, v, heads, extra)` runs the
+    rank-local route + attention over the heads the rank now holds (e.g. local_attention), and
+    return_heads sends the migrated heads' outputs home in the original head order.
+    Returns (o [B, N, H_local, d] in `local_heads` order, the balance_step record)."""
+    st = balance_step(L_h_local, local_heads, [q, k, v], rank, world, group=group, **policy)
+    q2, k2, v2 = st["tensors"]
+    o2 = compute(q2, k2, v2, st["local_heads"], st["extra"])
+    return return_heads(o2, st["local_heads"], list(local_heads), st["moves"], rank, group), st
 
 
 def bsa_route_intermediates(plan, workspace):

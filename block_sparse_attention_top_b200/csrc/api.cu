@@ -138,6 +138,7 @@ int bsa_plan_create(bsa_plan** out, int B, int H, int T, int Hs, int Ws,
     p->order = order; p->N = N; p->nb = nb; p->rows = (int64_t)B * H * nb;
     p->device = dev; p->num_sms = prop.multiProcessorCount;
     p->l2_bytes = prop.l2CacheSize; p->schedule = BSA_SCHED_L2_HEADS;
+    p->wait_ns = 4000000000ull;
     std::vector<int32_t> perm((size_t)N);
     token_order(T, Hs, Ws, order, perm.data());
     if (cudaMalloc(&p->d_perm, (size_t)N * sizeof(int32_t)) != cudaSuccess ||
@@ -172,6 +173,12 @@ int bsa_plan_set_schedule(bsa_plan* p, int schedule) {
     if (schedule != BSA_SCHED_L2_HEADS && schedule != BSA_SCHED_HEAVIEST_FIRST && schedule != BSA_SCHED_IN_ORDER)
         return BSA_EINVAL;
     p->schedule = schedule;
+    return BSA_OK;
+}
+
+int bsa_plan_set_wait_limit(bsa_plan* p, uint64_t ns) {
+    if (!p) return BSA_EINVAL;
+    p->wait_ns = ns;
     return BSA_OK;
 }
 
@@ -215,7 +222,8 @@ size_t bsa_workspace_size(const bsa_plan* p, int op) {
     if (!p) return 0;
     if (op == BSA_OP_ROUTE) return route_ws_layout(*p).total;
     if (op == BSA_OP_ATTN) return attn_ws_layout(*p).total;
-    if (op == BSA_OP_MASK || op == BSA_OP_AUGMENT) return mask_ws_bytes(*p);
+    if (op == BSA_OP_MASK) return mask_ws_bytes(*p) + stripe_ws_bytes(*p);
+    if (op == BSA_OP_AUGMENT) return mask_ws_bytes(*p);
     return 0;
 }
 
@@ -311,6 +319,22 @@ int bsa_mask_window_anchor(const bsa_plan* p, int radius_frames, int n_anchor, i
     if (int rc = check_ws(ws, ws_bytes, mask_ws_bytes(*p))) return rc;
     BSA_LAUNCH(launch_mask_window_anchor(*p, radius_frames, n_anchor, step, (int32_t*)ws, row_ptr, col_idx, col_cap,
                                          nnz, (cudaStream_t)stream));
+    return BSA_OK;
+}
+
+int bsa_mask_stripes_device(const bsa_plan* p, const int32_t* params, int32_t* row_ptr, int32_t* col_idx,
+                            int64_t col_cap, int64_t* nnz, void* ws, size_t ws_bytes, void* stream) {
+    if (!p || !params || !row_ptr || !nnz) return BSA_EINVAL;
+    if (col_cap < 0 || (col_cap > 0 && !col_idx)) return BSA_EINVAL;
+    if (misaligned(row_ptr, 4) || (col_idx && misaligned(col_idx, 4)) || misaligned(nnz, 8)) return BSA_EINVAL;
+    for (int h = 0; h < p->H; ++h)
+        if (params[6 * h + 0] < 0 || params[6 * h + 3] < 0) return BSA_EINVAL;   // widths
+    if (p->H > kMaxStripeHeads) return BSA_EUNSUPPORTED;
+    if (p->rows * p->nb > INT32_MAX) return BSA_EUNSUPPORTED;    // worst-case nnz must fit row_ptr (int32)
+    const size_t counts_bytes = mask_ws_bytes(*p);
+    if (int rc = check_ws(ws, ws_bytes, counts_bytes + stripe_ws_bytes(*p))) return rc;
+    BSA_LAUNCH(launch_mask_stripes(*p, params, (int32_t*)ws, (char*)ws + counts_bytes, row_ptr, col_idx, col_cap,
+                                   nnz, (cudaStream_t)stream));
     return BSA_OK;
 }
 

@@ -56,9 +56,12 @@
 // more than 2^4 (so 16 P <= 256 fits e4m3), PV is a kind::f8f6f4 MMA with
 // fp32 accumulation, and the epilogue writes O[:, c] * sigma_c / l.
 //
-// Every wait on an mbarrier spins on test_wait and is bounded (about 4 s); on
-// expiry the CTA records BSA_EDEVICE, raises a shared abort flag that stops
-// the other roles, drains its own tensor-core work and frees TMEM.
+// Every wait on an mbarrier in the main loops spins on test_wait and is
+// bounded (the plan's wait limit, 4 s by default); on expiry the CTA records
+// BSA_EDEVICE and raises a shared abort flag that stops the other roles.
+// Before TMEM is freed and the CTA returns, each TMA thread waits (with a
+// fixed 4 s bound) until every tile it issued has landed and each MMA thread
+// until its MMAs are complete.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -116,6 +119,7 @@ struct Params {
     int64_t npad;
     float scale_log2;
     const float* sigma;      // F8: per (head, channel) V scale, [B*H, D]
+    unsigned long long wait_ns;   // bound of every main-loop wait
 };
 
 __device__ __forceinline__ int item_index(int k, int cta, int grid) {
@@ -193,7 +197,7 @@ __device__ __forceinline__ float softmax_row_e4m3(const uint32_t* s, float scale
     return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-template <int D, bool F8>
+template <int D, bool F8, uint32_t kEvery>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const Params prm) {
@@ -204,14 +208,15 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar0 = sbase + L::offBar;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offMisc + 8);
+    volatile WaitCtl* ctl = reinterpret_cast<volatile WaitCtl*>(smem + L::offMisc);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offMisc + 16);
     float* m_pub = reinterpret_cast<float*>(smem + L::offPub);          // [2][128]
     float* l_pub = m_pub + 2 * kBlk;                                     // [2][128]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
-        *abort_flag = 0;
+        ctl->abort = 0;
+        ctl->limit_ns = prm.wait_ns;
         for (int i = 0; i < NBARS; ++i) {
             uint32_t count = 1;
             if (i == S_FREE0 || i == S_FREE0 + 1 || i == P_FULL0 || i == P_FULL0 + 1 || i == O_FREE)
@@ -243,7 +248,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (w.open(prm, cta, grid); w.ok && ok; w.next(prm, cta, grid), ++u) {
                 const int bh = w.r / nb;
                 if (kside && w.first()) {
-                    if (q_it > 0 && !(ok = mbar_wait(bar(Q_EMPTY), (q_it - 1) & 1, abort_flag))) break;
+                    if (q_it > 0 && !(ok = mbar_wait<kEvery>(bar(Q_EMPTY), (q_it - 1) & 1, ctl))) break;
                     mbar_expect_tx(bar(Q_FULL), L::kTile);
                     const int i = w.r % nb;
                     for (int s = 0; s < D / 64; ++s)
@@ -258,7 +263,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (kside) {
                     const int st = u % kKStages;
                     const uint32_t use = u / kKStages;
-                    if (use > 0 && !(ok = mbar_wait(bar(K_EMPTY0 + st), (use - 1) & 1, abort_flag))) break;
+                    if (use > 0 && !(ok = mbar_wait<kEvery>(bar(K_EMPTY0 + st), (use - 1) & 1, ctl))) break;
                     mbar_expect_tx(bar(K_FULL0 + st), L::kTile);
                     for (int s = 0; s < D / 64; ++s)
                         tma_load_2d(sbase + L::offK + st * L::kTile + s * kBlk * 128, &tmK, s * 64, y,
@@ -266,7 +271,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 } else {
                     const int st = u % kVStages;
                     const uint32_t use = u / kVStages;
-                    if (use > 0 && !(ok = mbar_wait(bar(V_EMPTY0 + st), (use - 1) & 1, abort_flag))) break;
+                    if (use > 0 && !(ok = mbar_wait<kEvery>(bar(V_EMPTY0 + st), (use - 1) & 1, ctl))) break;
                     mbar_expect_tx(bar(V_FULL0 + st), L::kVTile);
                     if constexpr (F8) {
                         // e4m3 tile of (head, block j): rows (bh * nb + j) * D .. + D, 128 keys each
@@ -279,7 +284,15 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                 }
             }
-            if (!ok) { *abort_flag = 1; record_error(prm.err, BSA_EDEVICE, -1); }
+            if (!ok) { ctl->abort = 1; record_error(prm.err, BSA_EDEVICE, -1); }
+            // every tile this thread issued lands before the CTA exits (the last
+            // load of each stage completes its phase; nothing is issued after it)
+            const uint32_t stages = kside ? kKStages : kVStages;
+            for (uint32_t st = 0; st < stages; ++st) {
+                const uint32_t loads = u > st ? (u - 1 - st) / stages + 1 : 0;
+                if (loads > 0) mbar_drain(bar((kside ? K_FULL0 : V_FULL0) + st), (loads - 1) & 1);
+            }
+            if (kside && q_it > 0) mbar_drain(bar(Q_FULL), (q_it - 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- QK issuer
@@ -290,14 +303,14 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             bool ok = true;
             for (qc.open(prm, cta, grid); qc.ok && ok; qc.next(prm, cta, grid), ++uq) {
                 if (qc.first()) {                            // this item's Q tile has landed
-                    if (!(ok = mbar_wait(bar(Q_FULL), q_it & 1, abort_flag))) break;
+                    if (!(ok = mbar_wait<kEvery>(bar(Q_FULL), q_it & 1, ctl))) break;
                     ++q_it;
                 }
                 // S[uq&1] = Q K_uq^T once the group has loaded S_{uq-2} from that buffer
                 const int sb = uq & 1;
-                if (uq >= 2 && !(ok = mbar_wait(bar(S_FREE0 + sb), ((uq - 2) >> 1) & 1, abort_flag))) break;
+                if (uq >= 2 && !(ok = mbar_wait<kEvery>(bar(S_FREE0 + sb), ((uq - 2) >> 1) & 1, ctl))) break;
                 const int st = uq % kKStages;
-                if (!(ok = mbar_wait(bar(K_FULL0 + st), (uq / kKStages) & 1, abort_flag))) break;
+                if (!(ok = mbar_wait<kEvery>(bar(K_FULL0 + st), (uq / kKStages) & 1, ctl))) break;
                 fence_after();
                 const uint32_t d_s = tmem + (sb ? kColS1 : kColS0);
 #pragma unroll
@@ -311,13 +324,12 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (qc.last()) commit(bar(Q_EMPTY));         // the Q tile may be replaced
             }
             if (!ok) {
-                *abort_flag = 1;
+                ctl->abort = 1;
                 record_error(prm.err, BSA_EDEVICE, -2);
             }
             // drain: everything this thread issued completes before TMEM is freed
             commit(bar(DRAIN_QK));
-            volatile int no_abort = 0;
-            mbar_wait(bar(DRAIN_QK), 0, &no_abort);
+            mbar_drain(bar(DRAIN_QK), 0);
         }
     } else if (warp == kPvWarp) {
         // ---------------------------------------------------------- PV issuer
@@ -329,11 +341,11 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (pc.open(prm, cta, grid); pc.ok && ok; pc.next(prm, cta, grid), ++up) {
                 // O (+)= P_up V_up; the first block of an item also waits for the
                 // previous item's epilogue to have read O
-                if (!(ok = mbar_wait(bar(P_FULL0 + (up & 1)), (up >> 1) & 1, abort_flag))) break;
-                if (pc.first() && pc.items > 1 && !(ok = mbar_wait(bar(O_FREE), (pc.items - 2) & 1, abort_flag)))
+                if (!(ok = mbar_wait<kEvery>(bar(P_FULL0 + (up & 1)), (up >> 1) & 1, ctl))) break;
+                if (pc.first() && pc.items > 1 && !(ok = mbar_wait<kEvery>(bar(O_FREE), (pc.items - 2) & 1, ctl)))
                     break;
                 const int st = up % kVStages;
-                if (!(ok = mbar_wait(bar(V_FULL0 + st), (up / kVStages) & 1, abort_flag))) break;
+                if (!(ok = mbar_wait<kEvery>(bar(V_FULL0 + st), (up / kVStages) & 1, ctl))) break;
                 fence_after();
                 const bool fresh = pc.first();
                 const uint32_t p_tmem = tmem + L::kColP + (up & 1) * (kBlk / 2);
@@ -356,12 +368,11 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (pc.last()) commit(bar(O_DONE));
             }
             if (!ok) {
-                *abort_flag = 1;
+                ctl->abort = 1;
                 record_error(prm.err, BSA_EDEVICE, -4);
             }
             commit(bar(DRAIN_PV));
-            volatile int no_abort = 0;
-            mbar_wait(bar(DRAIN_PV), 0, &no_abort);
+            mbar_drain(bar(DRAIN_PV), 0);
         }
     } else {
         // ------------------------------------------------------------- softmax
@@ -394,7 +405,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if ((int)(t & 1) != g) continue;
                 const int j = clamp_col(prm.col_idx[jj], nb);
                 const bool first = jj == beg, last = jj == end - 1;
-                if (!(ok = warp_wait(bar(S_FULL0 + g), (t >> 1) & 1, abort_flag))) break;
+                if (!(ok = warp_wait<kEvery>(bar(S_FULL0 + g), (t >> 1) & 1, ctl))) break;
                 fence_after();
                 uint32_t sv[kBlk];
 #pragma unroll
@@ -413,7 +424,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // running maximum from the previous block (the other group)
                 float m_prev = -INFINITY;
                 if (t > 0) {
-                    if (!(ok = warp_wait(bar(M_PUB0 + pub_other), ((t - 1) >> 1) & 1, abort_flag))) break;
+                    if (!(ok = warp_wait<kEvery>(bar(M_PUB0 + pub_other), ((t - 1) >> 1) & 1, ctl))) break;
                     m_prev = m_pub[other];
                 }
                 float m_use = m_prev, alpha = 1.f;
@@ -441,7 +452,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // phase of its own (a parity wait on a barrier still a phase behind
                 // would match its previous phase).
                 if (t >= 2) {
-                    if (!(ok = warp_wait(bar(PV_DONE0 + g), ((t - 2) >> 1) & 1, abort_flag))) break;
+                    if (!(ok = warp_wait<kEvery>(bar(PV_DONE0 + g), ((t - 2) >> 1) & 1, ctl))) break;
                     fence_after();
                 }
                 const bool any_rescale = __any_sync(0xffffffffu, rescale);
@@ -449,7 +460,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     // O must hold every earlier block before it is rescaled: PV_{t-1}
                     // done.  That barrier's previous phase (PV_{t-3}) has completed, as
                     // PV_{t-2} just did, so this occasional parity wait is exact.
-                    if (!(ok = warp_wait(bar(PV_DONE0 + (1 - g)), ((t - 1) >> 1) & 1, abort_flag))) break;
+                    if (!(ok = warp_wait<kEvery>(bar(PV_DONE0 + (1 - g)), ((t - 1) >> 1) & 1, ctl))) break;
                     fence_after();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
@@ -468,7 +479,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // running row sum
                 float l_prev = 0.f;
                 if (t > 0) {
-                    if (!(ok = warp_wait(bar(L_PUB0 + pub_other), ((t - 1) >> 1) & 1, abort_flag))) break;
+                    if (!(ok = warp_wait<kEvery>(bar(L_PUB0 + pub_other), ((t - 1) >> 1) & 1, ctl))) break;
                     l_prev = l_pub[other];
                 }
                 const float l = first ? rowsum : l_prev * alpha + rowsum;
@@ -480,7 +491,7 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                                              // for consecutive blocks may overtake
                 if (!last) continue;
                 // epilogue: the item's last PV, then O / l to the tokens' raster rows
-                if (!(ok = warp_wait(bar(O_DONE), (items - 1) & 1, abort_flag))) break;
+                if (!(ok = warp_wait<kEvery>(bar(O_DONE), (items - 1) & 1, ctl))) break;
                 fence_after();
                 const float inv = 1.f / l;
 #pragma unroll
@@ -509,7 +520,9 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 mbar_arrive(bar(O_FREE));
             }
         }
-        if (!ok) { *abort_flag = 1; record_error(prm.err, BSA_EDEVICE, -3); }
+        if (!ok) { ctl->abort = 1; record_error(prm.err, BSA_EDEVICE, -3); }
+        tmem_wait_st();                                  // no TMEM access of this warp outlives the loop
+        tmem_wait_ld();
     }
 
     fence_before();
@@ -520,9 +533,9 @@ k_attn_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     }
 }
 
-template <int D, bool F8>
-cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
-                   cudaStream_t s) {
+template <int D, bool F8, uint32_t kEvery>
+cudaError_t launch_t(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
+                     cudaStream_t s) {
     using L = PPLayout<D, F8>;
     const int64_t rows_total = (int64_t)p.B * p.H * p.nb * p.block;
     CUtensorMap mq, mk, mv;
@@ -530,11 +543,20 @@ cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void
         return cudaErrorInvalidValue;
     if (F8 ? !make_map_u8(&mv, vp, (int64_t)p.B * p.H * p.nb * D, D) : !make_map(&mv, vp, rows_total, D, kBlk))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_attn_pp<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_pp<D, F8, kEvery>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::kAlloc);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<int64_t>(p.num_sms, p.rows);
-    k_attn_pp<D, F8><<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, prm);
+    k_attn_pp<D, F8, kEvery><<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, prm);
     return cudaGetLastError();
+}
+
+// a wait limit below a millisecond: the variant that checks it at every probe
+template <int D, bool F8>
+cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
+                   cudaStream_t s) {
+    if (prm.wait_ns < 1000000ull) return launch_t<D, F8, 0>(p, qp, kp, vp, prm, s);
+    return launch_t<D, F8, 1023>(p, qp, kp, vp, prm, s);
 }
 
 }  // namespace
@@ -558,6 +580,7 @@ cudaError_t launch_attn_pp(const bsa_plan& p, const void* qp, const void* kp, co
     prm.npad = p.nb * p.block;
     prm.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
     prm.sigma = sigma;
+    prm.wait_ns = p.wait_ns;
     if (sigma) {                      // e4m3 V tiles at vp, scales at sigma
         if (p.d == 128) return launch<128, true>(p, qp, kp, vp, prm, s);
         return launch<64, true>(p, qp, kp, vp, prm, s);

@@ -31,10 +31,12 @@
 // SM's whole shared-memory bandwidth at full MMA rate.  TMEM columns:
 // S0 [0,128) S1 [128,256) O [256,384) Q [384,448).
 //
-// Every wait on an mbarrier spins on test_wait and is bounded (about 4 s of
-// %globaltimer, checked every 1024 probes); on expiry
-// the CTA records BSA_EDEVICE, raises a shared abort flag that stops the other
-// roles, drains its own tensor-core work and frees TMEM before returning.
+// Every wait on an mbarrier in the main loops spins on test_wait and is
+// bounded (the plan's wait limit, 4 s of %globaltimer by default); on expiry
+// the CTA records BSA_EDEVICE and raises a shared abort flag that stops the
+// other roles.  Before TMEM is freed and the CTA returns, each TMA thread
+// waits (with a fixed 4 s bound) until every tile it issued has landed and
+// the MMA thread until its MMAs are complete.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -111,6 +113,7 @@ struct Params {
     int N, H, nb, rows;
     int64_t npad;
     float scale_log2;
+    unsigned long long wait_ns;   // bound of every main-loop wait
 };
 
 // Work item sequence of this CTA: zig-zag over the heaviest-first list.
@@ -120,7 +123,7 @@ __device__ __forceinline__ int item_index(int k, int cta, int grid) {
 
 __device__ __forceinline__ bool valid_col(int j, int nb) { return j >= 0 && j < nb; }
 
-template <int D, int BLK>
+template <int D, int BLK, uint32_t kEvery>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const Params prm) {
@@ -133,14 +136,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar0 = sbase + L::offBar;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offMisc + 8);
+    volatile WaitCtl* ctl = reinterpret_cast<volatile WaitCtl*>(smem + L::offMisc);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offMisc + 16);
     float* xchg = reinterpret_cast<float*>(smem + L::offXchg);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
-        *abort_flag = 0;
+        ctl->abort = 0;
+        ctl->limit_ns = prm.wait_ns;
         for (int i = 0; i < B_COUNT; ++i)
             mbar_init(bar(i), i == B_PFULL ? 32u * kSoftmaxWarps : (i >= B_PAIR0 ? 64u : 1u));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -182,7 +186,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (end <= beg) continue;                    // no key block: no Q either
                 const int bh = r / nb, i = r % nb;
                 if (kside) {
-                    if (q_it > 0 && !(ok = mbar_wait(bar(B_QEMPTY), (q_it - 1) & 1, abort_flag))) break;
+                    if (q_it > 0 && !(ok = mbar_wait<kEvery>(bar(B_QEMPTY), (q_it - 1) & 1, ctl))) break;
                     mbar_expect_tx(bar(B_QFULL), BLK * D * 2);
                     for (int s = 0; s < D / 64; ++s)
                         tma_load_2d(sbase + L::offQ + s * kTileM * 128, &tmQ, s * 64,
@@ -201,7 +205,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     if (kside) {
                         const int st = kv_it % kKStages;
                         const uint32_t use = kv_it / kKStages;
-                        if (use > 0 && !(ok = mbar_wait(bar(B_KEMPTY0 + st), (use - 1) & 1, abort_flag))) break;
+                        if (use > 0 && !(ok = mbar_wait<kEvery>(bar(B_KEMPTY0 + st), (use - 1) & 1, ctl))) break;
                         mbar_expect_tx(bar(B_KFULL0 + st), L::kKV);
                         for (int s = 0; s < D / 64; ++s)
                             tma_load_2d(sbase + L::offK + st * L::kKV + s * BLK * 128, &tmK, s * 64, y,
@@ -209,7 +213,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     } else {
                         const int st = kv_it % kVStages;
                         const uint32_t use = kv_it / kVStages;
-                        if (use > 0 && !(ok = mbar_wait(bar(B_VEMPTY0 + st), (use - 1) & 1, abort_flag))) break;
+                        if (use > 0 && !(ok = mbar_wait<kEvery>(bar(B_VEMPTY0 + st), (use - 1) & 1, ctl))) break;
                         mbar_expect_tx(bar(B_VFULL0 + st), L::kKV);
                         for (int s = 0; s < D / 64; ++s)
                             tma_load_2d(sbase + L::offV + st * L::kKV + s * BLK * 128, &tmV, s * 64, y,
@@ -218,7 +222,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     ++kv_it;
                 }
             }
-            if (!ok) { *abort_flag = 1; record_error(prm.err, BSA_EDEVICE, -1); }
+            if (!ok) { ctl->abort = 1; record_error(prm.err, BSA_EDEVICE, -1); }
+            // every tile this thread issued lands before the CTA exits (the last
+            // load of each stage completes its phase; nothing is issued after it)
+            const uint32_t stages = kside ? kKStages : kVStages;
+            for (uint32_t st = 0; st < stages; ++st) {
+                const uint32_t loads = kv_it > st ? (kv_it - 1 - st) / stages + 1 : 0;
+                if (loads > 0) mbar_drain(bar((kside ? B_KFULL0 : B_VFULL0) + st), (loads - 1) & 1);
+            }
+            if (kside && q_it > 0) mbar_drain(bar(B_QFULL), (q_it - 1) & 1);
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------------- MMA
@@ -229,9 +241,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             bool ok = true;
             // O += P V for kv iteration `it`; P sits in TMEM buffer it&1
             auto issue_pv = [&](uint32_t it, bool first) -> bool {
-                if (!mbar_wait(bar(B_PFULL), pv_it & 1, abort_flag)) return false;
+                if (!mbar_wait<kEvery>(bar(B_PFULL), pv_it & 1, ctl)) return false;
                 const int st = it % kVStages;
-                if (!mbar_wait(bar(B_VFULL0 + st), (it / kVStages) & 1, abort_flag)) return false;
+                if (!mbar_wait<kEvery>(bar(B_VFULL0 + st), (it / kVStages) & 1, ctl)) return false;
                 fence_after();
                 const uint32_t p_tmem = tmem + ((it & 1) ? kColS1 : kColS0);   // P overwrote S(it)
 #pragma unroll
@@ -250,7 +262,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const int r = prm.work[idx];
                 const int beg = prm.row_ptr[r], end = prm.row_ptr[r + 1];
                 if (end <= beg) continue;
-                if (!(ok = mbar_wait(bar(B_QFULL), q_it & 1, abort_flag))) break;
+                if (!(ok = mbar_wait<kEvery>(bar(B_QFULL), q_it & 1, ctl))) break;
                 ++q_it;
                 // Q -> TMEM (16 columns of bf16 per copy), then its shared buffer is free.
                 // The previous item's QKs have completed: the last PV issued above waited
@@ -272,7 +284,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     // S buffer kv_it&1 is free: the softmax warps read S(kv_it-2) before the
                     // P_FULL arrival this thread waited on for PV(kv_it-2), and that PV, which
                     // read P from the same columns, was issued earlier by this thread.
-                    if (!(ok = mbar_wait(bar(B_KFULL0 + st), (kv_it / kKStages) & 1, abort_flag))) break;
+                    if (!(ok = mbar_wait<kEvery>(bar(B_KFULL0 + st), (kv_it / kKStages) & 1, ctl))) break;
                     fence_after();
                     const uint32_t d_s = tmem + ((kv_it & 1) ? kColS1 : kColS0);
 #pragma unroll
@@ -290,13 +302,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (local > 0 && !(ok = issue_pv(kv_it - 1, local == 1))) break;
             }
             if (!ok) {
-                *abort_flag = 1;
+                ctl->abort = 1;
                 record_error(prm.err, BSA_EDEVICE, -2);
             }
             // drain: everything this thread issued completes before TMEM is freed
             commit(bar(B_DRAIN));
-            volatile int no_abort = 0;
-            mbar_wait(bar(B_DRAIN), 0, &no_abort);
+            mbar_drain(bar(B_DRAIN), 0);
         }
     } else {
         // ------------------------------------------------------------- softmax
@@ -326,7 +337,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (!valid_col(j, nb)) continue;
                 const int sb = kv_it & 1;
                 const uint32_t s_col = sb ? kColS1 : kColS0;
-                if (!(ok = warp_wait(bar(B_SFULL0 + sb), (kv_it >> 1) & 1, abort_flag))) break;
+                if (!(ok = warp_wait<kEvery>(bar(B_SFULL0 + sb), (kv_it >> 1) & 1, ctl))) break;
                 fence_after();
                 // padding keys of a ragged last block
                 const int valid_keys = prm.N - j * BLK;
@@ -346,7 +357,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 float* xs = xchg + sb * 2 * kTileM;
                 xs[half * kTileM + row] = lmax;
                 mbar_arrive(bar(B_PAIR0 + quad));
-                if (!(ok = warp_wait(bar(B_PAIR0 + quad), pairs & 1, abort_flag))) break;
+                if (!(ok = warp_wait<kEvery>(bar(B_PAIR0 + quad), pairs & 1, ctl))) break;
                 ++pairs;
                 const float mx = fmaxf(lmax, xs[(1 - half) * kTileM + row]) * prm.scale_log2;
                 float alpha = 1.f;
@@ -373,7 +384,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // the previous PV must be done before O is rescaled; waiting on it every
                 // block keeps at most one PV completion outstanding for this warp
                 if (local > 0) {
-                    if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
+                    if (!(ok = warp_wait<kEvery>(bar(B_PVDONE), pv_it & 1, ctl))) break;
                     ++pv_it;
                     fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
@@ -402,13 +413,13 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             }
             // epilogue: last PV of the item; the two partial row sums meet in shared
             // memory (slots alternate by item; a bounded mbarrier pairs the two warps)
-            if (!(ok = warp_wait(bar(B_PVDONE), pv_it & 1, abort_flag))) break;
+            if (!(ok = warp_wait<kEvery>(bar(B_PVDONE), pv_it & 1, ctl))) break;
             ++pv_it;
             fence_after();
             float* ls = xchg + 4 * kTileM + (items & 1) * 2 * kTileM;
             ls[half * kTileM + row] = l;
             mbar_arrive(bar(B_PAIR0 + quad));
-            if (!(ok = warp_wait(bar(B_PAIR0 + quad), pairs & 1, abort_flag))) break;
+            if (!(ok = warp_wait<kEvery>(bar(B_PAIR0 + quad), pairs & 1, ctl))) break;
             ++pairs;
             ++items;
             const float inv = 1.f / (l + ls[(1 - half) * kTileM + row]);
@@ -431,7 +442,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             }
             fence_before();
         }
-        if (!ok) { *abort_flag = 1; record_error(prm.err, BSA_EDEVICE, -3); }
+        if (!ok) { ctl->abort = 1; record_error(prm.err, BSA_EDEVICE, -3); }
+        tmem_wait_st();                                  // no TMEM access of this warp outlives the loop
+        tmem_wait_ld();
     }
 
     fence_before();
@@ -443,20 +456,29 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 }
 
 // ----------------------------------------------------------------- host side
-template <int D, int BLK>
-cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
-                   cudaStream_t s) {
+template <int D, int BLK, uint32_t kEvery>
+cudaError_t launch_t(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
+                     cudaStream_t s) {
     using L = Smem<D, BLK>;
     const int64_t rows_total = (int64_t)p.B * p.H * p.nb * p.block;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, qp, rows_total, D, BLK) || !make_map(&mk, kp, rows_total, D, BLK) ||
         !make_map(&mv, vp, rows_total, D, BLK))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D, BLK, kEvery>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::kAlloc);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<int64_t>(p.num_sms, p.rows);
-    k_attn_tc<D, BLK><<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, prm);
+    k_attn_tc<D, BLK, kEvery><<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, prm);
     return cudaGetLastError();
+}
+
+// a wait limit below a millisecond: the variant that checks it at every probe
+template <int D, int BLK>
+cudaError_t launch(const bsa_plan& p, const void* qp, const void* kp, const void* vp, const Params& prm,
+                   cudaStream_t s) {
+    if (prm.wait_ns < 1000000ull) return launch_t<D, BLK, 0>(p, qp, kp, vp, prm, s);
+    return launch_t<D, BLK, 1023>(p, qp, kp, vp, prm, s);
 }
 
 }  // namespace
@@ -478,10 +500,12 @@ cudaError_t launch_attn_tc(const bsa_plan& p, const void* qp, const void* kp, co
     prm.rows = (int)p.rows;
     prm.npad = p.nb * p.block;
     prm.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
+    prm.wait_ns = p.wait_ns;
     if (p.d == 128 && p.block == 128) return launch<128, 128>(p, qp, kp, vp, prm, s);
     if (p.d == 128 && p.block == 64) return launch<128, 64>(p, qp, kp, vp, prm, s);
     if (p.d == 64 && p.block == 128) return launch<64, 128>(p, qp, kp, vp, prm, s);
     return launch<64, 64>(p, qp, kp, vp, prm, s);
 }
+
 
 }  // namespace bsa

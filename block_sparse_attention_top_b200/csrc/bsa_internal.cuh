@@ -14,6 +14,7 @@ struct bsa_plan {
     int num_sms;
     int64_t l2_bytes;    // the device's L2 size (sizes the head groups of BSA_SCHED_L2_HEADS)
     int schedule;        // BSA_SCHED_*: order of the attention work list
+    unsigned long long wait_ns;   // bound of the attention kernels' main-loop waits
     int32_t* d_perm;     // [N] raster index at reordered position
     int32_t* d_err;      // [4]: status, detail, spare, spare
 };
@@ -34,6 +35,8 @@ RouteWs route_ws_layout(const bsa_plan& p);
 // ---- attention workspace layout ----
 // ---- mask workspace: per-row counts ----
 inline size_t mask_ws_bytes(const bsa_plan& p) { return align_up((size_t)p.rows * sizeof(int32_t)); }
+// BSA_OP_MASK: the counts plus, for the stripe producer, the block ranges
+size_t stripe_ws_bytes(const bsa_plan& p);
 
 struct AttnWs {
     size_t qp, kp, vp, work, hist, bins, counter, vscale, grank, total;
@@ -64,6 +67,13 @@ cudaError_t launch_mask_window_anchor(const bsa_plan& p, int radius, int n_ancho
                                       int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, int64_t* nnz,
                                       cudaStream_t s);
 constexpr int kMaxMaskAnchors = 64;
+// Stripe masks on the device: per-head parameters travel in the launch (at
+// most kMaxStripeHeads heads); block frame/row ranges live in the workspace
+// behind the per-row counts.
+constexpr int kMaxStripeHeads = 160;
+size_t stripe_ws_bytes(const bsa_plan& p);
+cudaError_t launch_mask_stripes(const bsa_plan& p, const int32_t* params, int32_t* counts, void* ranges_ws,
+                                int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, int64_t* nnz, cudaStream_t s);
 cudaError_t launch_augment(const bsa_plan& p, const int32_t* row_ptr, const uint16_t* order, const int32_t* extra,
                            int32_t* counts, int32_t* row_ptr_out, int32_t* col_idx_out, int64_t col_cap,
                            float* L_h_out, int64_t* nnz_out, cudaStream_t s);

@@ -22,11 +22,16 @@ namespace bsa {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Pooling: one CTA per (query/key tensor, batch, block, chunk of the H*d row).
-// Each thread owns 8 (bf16) or 4 (fp32) consecutive elements of a token row
-// (one 16-byte load per token) and sums them over the block's tokens.
+// Pooling: one CTA per (query/key tensor, batch, block, 64 chunks of the H*d
+// row).  Thread (g, c) owns the 16-byte chunk c (8 bf16 or 4 fp32 values) of
+// a token row and sums it over token group g (tokens g, g+4, g+8, ... of the
+// block, 16 loads in flight); the four partial sums meet in shared memory.
+// Sums of bf16 (or fp32) values in fp64 are exact here, so the order of the
+// partial sums does not change the result.
 // ---------------------------------------------------------------------------
-constexpr int kPoolThreads = 256;
+constexpr int kPoolChunks = 64;              // 16-byte chunks per CTA
+constexpr int kPoolGroups = 4;               // token groups per chunk
+constexpr int kPoolThreads = kPoolChunks * kPoolGroups;
 constexpr int kPoolUnroll = 16;
 
 template <typename T> struct Vec16;
@@ -57,6 +62,7 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
        double* __restrict__ qbar, double* __restrict__ kbar, int N, int H, int d, int block, int nb) {
     constexpr int V = Vec16<T>::n;
     __shared__ int32_t s_tok[128];
+    __shared__ double part[kPoolGroups - 1][kPoolChunks][V];
     const int i = blockIdx.x;
     const int which = blockIdx.z & 1;
     const int b = blockIdx.z >> 1;
@@ -68,34 +74,48 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
     __syncthreads();
 
     const int hd = H * d;
-    const int c = blockIdx.y * blockDim.x + threadIdx.x;   // 16-byte chunk within the row
-    if (c * V >= hd) return;
+    const int g = threadIdx.x / kPoolChunks;
+    const int c = blockIdx.y * kPoolChunks + threadIdx.x % kPoolChunks;   // 16-byte chunk within the row
+    const bool live = c * V < hd;
     const uint4* base = reinterpret_cast<const uint4*>(x + (size_t)b * N * hd) + c;
     const size_t row_stride = (size_t)hd / V;              // in uint4
 
     double acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.0;
-    int t = 0;
-    for (; t + kPoolUnroll <= m; t += kPoolUnroll) {
-        uint4 u[kPoolUnroll];
+    if (live) {
+        int t = g;
+        for (; t + kPoolGroups * (kPoolUnroll - 1) < m; t += kPoolGroups * kPoolUnroll) {
+            uint4 u[kPoolUnroll];
 #pragma unroll
-        for (int r = 0; r < kPoolUnroll; ++r) u[r] = __ldg(base + (size_t)s_tok[t + r] * row_stride);
+            for (int r = 0; r < kPoolUnroll; ++r)
+                u[r] = __ldg(base + (size_t)s_tok[t + kPoolGroups * r] * row_stride);
 #pragma unroll
-        for (int r = 0; r < kPoolUnroll; ++r) {
+            for (int r = 0; r < kPoolUnroll; ++r) {
+                double w[V];
+                Vec16<T>::widen(u[r], w);
+#pragma unroll
+                for (int e = 0; e < V; ++e) acc[e] += w[e];
+            }
+        }
+        for (; t < m; t += kPoolGroups) {
+            const uint4 u = __ldg(base + (size_t)s_tok[t] * row_stride);
             double w[V];
-            Vec16<T>::widen(u[r], w);
+            Vec16<T>::widen(u, w);
 #pragma unroll
             for (int e = 0; e < V; ++e) acc[e] += w[e];
         }
     }
-    for (; t < m; ++t) {
-        const uint4 u = __ldg(base + (size_t)s_tok[t] * row_stride);
-        double w[V];
-        Vec16<T>::widen(u, w);
+    if (g > 0) {
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] += w[e];
+        for (int e = 0; e < V; ++e) part[g - 1][threadIdx.x % kPoolChunks][e] = acc[e];
     }
+    __syncthreads();
+    if (g > 0 || !live) return;
+#pragma unroll
+    for (int u = 0; u < kPoolGroups - 1; ++u)
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += part[u][threadIdx.x][e];
     const int h = (c * V) / d;
     const int dd = (c * V) % d;
     double* dst = out + (((size_t)b * H + h) * nb + i) * d + dd;
@@ -180,6 +200,101 @@ k_scores(const double* __restrict__ qbar, const double* __restrict__ kbar, doubl
             const int j = j0 + tx + 16 * v;
             if (j < nb) out[(size_t)i * nb + j] = acc[u][v] * scale;
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Scores on the FP64 MMA path (mma.sync m8n8k4 .f64: fp64 products and sums,
+// the same precision as the FMA kernel above, a different summation order).
+// CTA tile 64 x 64 of one head, 4 warps of 32 x 32 (4 x 4 tiles of 8 x 8);
+// Qbar and Kbar staged in slices of 16 along d, double-buffered.  Fragments
+// of m8n8k4: A (8x4) a0 = A[lane/4][lane%4]; B (4x8) b0 = B[lane%4][lane/4];
+// C (8x8) c0, c1 = C[lane/4][2*(lane%4) + {0,1}].
+// ---------------------------------------------------------------------------
+constexpr int kMT = 64;                  // CTA tile (rows and columns)
+constexpr int kMK = 16;                  // d slice
+constexpr int kMLd = kMK + 1;            // padded shared row (doubles)
+
+__device__ __forceinline__ void dmma(double& c0, double& c1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                 : "+d"(c0), "+d"(c1)
+                 : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(128)
+k_scores_mma(const double* __restrict__ qbar, const double* __restrict__ kbar, double* __restrict__ S, int nb,
+             int d, double scale) {
+    __shared__ double As[2][kMT][kMLd];
+    __shared__ double Bs[2][kMT][kMLd];
+    const int bh = blockIdx.z;
+    const int i0 = blockIdx.y * kMT, j0 = blockIdx.x * kMT;
+    const double* Q = qbar + (size_t)bh * nb * d;
+    const double* K = kbar + (size_t)bh * nb * d;
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int g = lane >> 2, t = lane & 3;
+    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+    double acc[4][4][2];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
+    // slice loads: 64 rows x 16 doubles per operand = 512 double2, 4 per thread
+    double2 ra[4], rb[4];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            const int e = tid + 128 * l, r = e / (kMK / 2), c2 = e % (kMK / 2);
+            const double2 z = make_double2(0.0, 0.0);
+            ra[l] = (i0 + r < nb) ? *reinterpret_cast<const double2*>(Q + (size_t)(i0 + r) * d + k0 + 2 * c2) : z;
+            rb[l] = (j0 + r < nb) ? *reinterpret_cast<const double2*>(K + (size_t)(j0 + r) * d + k0 + 2 * c2) : z;
+        }
+    };
+    auto stash = [&](int buf) {
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            const int e = tid + 128 * l, r = e / (kMK / 2), c2 = e % (kMK / 2);
+            As[buf][r][2 * c2] = ra[l].x;
+            As[buf][r][2 * c2 + 1] = ra[l].y;
+            Bs[buf][r][2 * c2] = rb[l].x;
+            Bs[buf][r][2 * c2 + 1] = rb[l].y;
+        }
+    };
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < d; k0 += kMK) {
+        const bool more = k0 + kMK < d;
+        if (more) fetch(k0 + kMK);                    // in flight while this slice is multiplied
+#pragma unroll
+        for (int ks = 0; ks < kMK / 4; ++ks) {
+            double av[4], bv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                av[u] = As[buf][wm + 8 * u + g][4 * ks + t];
+                bv[u] = Bs[buf][wn + 8 * u + g][4 * ks + t];
+            }
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) dmma(acc[mt][nt][0], acc[mt][nt][1], av[mt], bv[nt]);
+        }
+        if (more) stash(buf ^ 1);                     // the other buffer was last read one slice ago
+        __syncthreads();
+        buf ^= 1;
+    }
+    double* out = S + (size_t)bh * nb * nb;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+        const int i = i0 + wm + 8 * mt + g;
+        if (i >= nb) continue;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int j = j0 + wn + 8 * nt + 2 * t + e;
+                if (j < nb) out[(size_t)i * nb + j] = acc[mt][nt][e] * scale;
+            }
     }
 }
 
@@ -442,6 +557,154 @@ k_route_cta(const double* __restrict__ S, int nb, double p, int k_floor,
 }
 
 // ---------------------------------------------------------------------------
+// Row routing by an exact bucket sort (rows of more than 256 blocks): one
+// 128-thread CTA per row.  Each score goes to bucket floor((max - s) * NB /
+// (max - min)) -- monotone in s, so every key of a bucket sorts after every
+// key of a lower bucket -- the buckets are laid out by a shared-memory count
+// and exclusive scan, and each key takes its place inside its bucket by
+// counting the smaller keys there (the same 64-bit keys as above: s
+// descending, j ascending, so the result is the exact order).  P, the
+// inclusive cumulative mass (a block scan in sorted order) and the Top-p cut
+// follow in fp64, as in the warp kernel.
+// ---------------------------------------------------------------------------
+constexpr int kBucketThreads = 128;
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < kBucketThreads / 32; ++w) t += red[w];
+    return t;
+}
+__device__ __forceinline__ double block_max(double v, double* red) {
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    double t = red[0];
+#pragma unroll
+    for (int w = 1; w < kBucketThreads / 32; ++w) t = fmax(t, red[w]);
+    return t;
+}
+
+// dynamic shared memory: keys [nb] u64, placed [nb] u64, count [NB] int, start [NB] int
+__global__ void __launch_bounds__(kBucketThreads)
+k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_floor,
+               uint16_t* __restrict__ sorted, int32_t* __restrict__ counts) {
+    extern __shared__ unsigned long long bsm[];
+    unsigned long long* keys = bsm;
+    unsigned long long* placed = bsm + nb;
+    int* cnt = reinterpret_cast<int*>(bsm + 2 * nb);
+    int* start = cnt + NB;
+    __shared__ double red[kBucketThreads / 32];
+    __shared__ int s_first;
+    const int tid = threadIdx.x;
+    const size_t r = blockIdx.x;
+    const double* row = S + r * nb;
+
+    double mx = -INFINITY, mn = INFINITY;
+    for (int j = tid; j < nb; j += kBucketThreads) {
+        const double sv = row[j];
+        mx = fmax(mx, sv);
+        mn = fmin(mn, sv);
+        keys[j] = desc_key(sv, j);
+    }
+    for (int b = tid; b < NB; b += kBucketThreads) cnt[b] = 0;
+    if (tid == 0) s_first = nb;
+    mx = block_max(mx, red);
+    mn = -block_max(-mn, red);
+    const double width = mx - mn;
+    const double to_bucket = width > 0.0 ? (double)NB / width : 0.0;
+    // bucket counts; each key keeps its arrival slot only to be placed somewhere in its bucket
+    double zpart = 0.0;
+    for (int j = tid; j < nb; j += kBucketThreads) {
+        const double sv = key_score(keys[j]);
+        zpart += exp(sv - mx);
+        const int b = min(NB - 1, (int)((mx - row[j]) * to_bucket));
+        atomicAdd(&cnt[b], 1);
+    }
+    const double z = block_sum(zpart, red);
+    __syncthreads();
+    // exclusive scan of the counts (NB / 128 per thread, then across the block)
+    {
+        const int per = NB / kBucketThreads;
+        const int lo = tid * per;
+        int run = 0;
+        for (int u = 0; u < per; ++u) run += cnt[lo + u];
+        int incl = run;
+        const int lane = tid % 32, wid = tid / 32;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        __shared__ int wsum[kBucketThreads / 32];
+        if (lane == 31) wsum[wid] = incl;
+        __syncthreads();
+        int off = incl - run;
+        for (int w = 0; w < wid; ++w) off += wsum[w];
+        for (int u = 0; u < per; ++u) {
+            start[lo + u] = off;
+            off += cnt[lo + u];
+            cnt[lo + u] = 0;                      // reused as the fill cursor
+        }
+    }
+    __syncthreads();
+    for (int j = tid; j < nb; j += kBucketThreads) {
+        const int b = min(NB - 1, (int)((mx - row[j]) * to_bucket));
+        placed[start[b] + atomicAdd(&cnt[b], 1)] = keys[j];
+    }
+    __syncthreads();
+    // each key's final place: its bucket's start + the number of smaller keys in the bucket
+    for (int q = tid; q < nb; q += kBucketThreads) {
+        const unsigned long long key = placed[q];
+        const int b = min(NB - 1, (int)((mx - row[(int)(key & kJMask)]) * to_bucket));
+        const int b0 = start[b], b1 = b0 + cnt[b];
+        int rank = b0;
+        for (int u = b0; u < b1; ++u) rank += placed[u] < key;
+        keys[rank] = key;
+    }
+    __syncthreads();
+    // P in sorted order, inclusive cumulative mass (contiguous chunks per thread), first n with C_n >= p
+    const int per = (nb + kBucketThreads - 1) / kBucketThreads;
+    const int q0 = tid * per, q1 = min(nb, q0 + per);
+    double run = 0.0;
+    for (int q = q0; q < q1; ++q) run += exp(key_score(keys[q]) - mx) / z;
+    double incl = run;
+    const int lane = tid % 32, wid = tid / 32;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) red[wid] = incl;
+    __syncthreads();
+    double c = incl - run;
+    for (int w = 0; w < wid; ++w) c += red[w];
+    int first = nb;
+    for (int q = q0; q < q1; ++q) {
+        c += exp(key_score(keys[q]) - mx) / z;
+        if (c >= p) { first = q + 1; break; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    if (lane == 0 && first < nb) atomicMin(&s_first, first);
+    __syncthreads();
+    const int n_p = p >= 1.0 ? nb : s_first;
+    const int n_i = min(nb, max(k_floor, n_p));
+    uint16_t* dst = sorted + r * nb;
+    for (int q = tid; q < nb; q += kBucketThreads) dst[q] = (uint16_t)(keys[q] & kJMask);   // the full importance order
+    if (tid == 0) counts[r] = n_i;
+}
+
+// ---------------------------------------------------------------------------
 // CSR: single-CTA exclusive scan of the counts, then a row-parallel copy.
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 1024;
@@ -513,14 +776,14 @@ cudaError_t launch_pool(const bsa_plan& p, const void* q, const void* k, int dty
                         double* qbar, double* kbar, cudaStream_t s) {
     const int V = dtype == BSA_BF16 ? 8 : 4;
     const int chunks = (p.H * p.d) / V;
-    const int threads = chunks >= kPoolThreads ? kPoolThreads : (chunks + 31) / 32 * 32;
-    dim3 grid((unsigned)p.nb, (unsigned)((chunks + threads - 1) / threads), (unsigned)(2 * p.B));
+    dim3 grid((unsigned)p.nb, (unsigned)((chunks + kPoolChunks - 1) / kPoolChunks), (unsigned)(2 * p.B));
     if (dtype == BSA_BF16)
-        k_pool<__nv_bfloat16><<<grid, threads, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                       p.d_perm, qbar, kbar, (int)p.N, p.H, p.d, p.block, (int)p.nb);
+        k_pool<__nv_bfloat16><<<grid, kPoolThreads, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                            p.d_perm, qbar, kbar, (int)p.N, p.H, p.d, p.block,
+                                                            (int)p.nb);
     else
-        k_pool<float><<<grid, threads, 0, s>>>((const float*)q, (const float*)k, p.d_perm, qbar, kbar,
-                                               (int)p.N, p.H, p.d, p.block, (int)p.nb);
+        k_pool<float><<<grid, kPoolThreads, 0, s>>>((const float*)q, (const float*)k, p.d_perm, qbar, kbar,
+                                                    (int)p.N, p.H, p.d, p.block, (int)p.nb);
     return cudaGetLastError();
 }
 
@@ -541,6 +804,12 @@ cudaError_t launch_scores_tm(const bsa_plan& p, const double* qbar, const double
 cudaError_t launch_scores(const bsa_plan& p, const double* qbar, const double* kbar, double* scores,
                           cudaStream_t s) {
     const double scale = 1.0 / sqrt((double)p.d);
+    if (p.d % kMK == 0) {
+        const int t = (int)((p.nb + kMT - 1) / kMT);
+        dim3 grid(t, t, (unsigned)(p.B * p.H));
+        k_scores_mma<<<grid, 128, 0, s>>>(qbar, kbar, scores, (int)p.nb, p.d, scale);
+        return cudaGetLastError();
+    }
     const int64_t t128 = (p.nb + 127) / 128;
     if (t128 * t128 * p.B * p.H >= 2 * p.num_sms) return launch_scores_tm<128>(p, qbar, kbar, scores, s, scale);
     return launch_scores_tm<64>(p, qbar, kbar, scores, s, scale);
@@ -562,23 +831,15 @@ cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pv
         }
         return cudaGetLastError();
     }
-    const int E = nbp / kCtaSortThreads;
-    const size_t smem = (size_t)nbp * sizeof(unsigned long long);
-    auto run = [&](auto kern) -> cudaError_t {
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-        }
-        kern<<<(unsigned)p.rows, kCtaSortThreads, smem, s>>>(scores, nb, pval, k_floor, sorted, counts);
-        return cudaGetLastError();
-    };
-    switch (E) {
-        case 2: return run(k_route_cta<2>);
-        case 4: return run(k_route_cta<4>);
-        case 8: return run(k_route_cta<8>);
-        case 16: return run(k_route_cta<16>);
-        default: return run(k_route_cta<32>);
+    // exact bucket sort: NB = 2 * nbp buckets, at most 8192 (a multiple of the block size)
+    const int NB = 2 * nbp < 8192 ? 2 * nbp : 8192;
+    const size_t smem = (size_t)2 * nb * sizeof(unsigned long long) + (size_t)2 * NB * sizeof(int);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_route_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
     }
+    k_route_bucket<<<(unsigned)p.rows, kBucketThreads, smem, s>>>(scores, nb, NB, pval, k_floor, sorted, counts);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_scan_counts(const bsa_plan& p, const int32_t* counts, int32_t* row_ptr, float* L_h,

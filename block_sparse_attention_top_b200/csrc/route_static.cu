@@ -21,6 +21,10 @@ constexpr int kMaxDevices = 64;
 // is only a stand-in.  The device address is fetched once per device below.
 static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
 
+// Cached per device for the life of the process.  The address belongs to the
+// device's primary context: a cudaDeviceReset (or anything else that destroys
+// that context) leaves it stale, and the header tells callers not to route
+// through this entry point after such a reset.
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 

@@ -46,23 +46,43 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __noinline__ inline bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// Control block of a CTA's bounded waits (in shared memory): the abort flag
+// every role raises when it gives up, and the time limit of a wait.  Only the
+// slow path reads it, every kEvery + 1 probes, so the waiting code carries no
+// extra live values.  kEvery = 1023 in normal launches; a launch with a limit
+// below a millisecond uses kEvery = 0 (every probe), so a zero limit gives up
+// at the first probe that fails.
+struct WaitCtl {
+    int abort;
+    int pad;
+    unsigned long long limit_ns;
+};
+template <uint32_t kEvery>
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl) {
     const unsigned long long t0 = globaltimer();
     for (uint32_t n = 1;; ++n) {
         if (mbar_test(bar, parity)) return true;
-        if ((n & 1023u) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > kTimeoutNs) return false;
+        if ((n & kEvery) == 0) {
+            if (ctl->abort) return false;
+            if (globaltimer() - t0 >= ctl->limit_ns) return false;
         }
     }
 }
 // Bounded wait: false if the abort flag is raised or the time limit passes.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, abort_flag);
+template <uint32_t kEvery = 1023>
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl) {
+    return mbar_test(bar, parity) || mbar_wait_slow<kEvery>(bar, parity, ctl);
 }
 // Warp-uniform bounded wait (every lane polls; all lanes agree on the outcome).
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+template <uint32_t kEvery = 1023>
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl) {
+    return __all_sync(0xffffffffu, mbar_wait<kEvery>(bar, parity, ctl));
+}
+// A wait that only the time limit ends (4 s; no abort flag): for draining a
+// CTA's own copies and MMAs before it exits.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+    WaitCtl own{0, 0, kTimeoutNs};
+    return mbar_wait<1023>(bar, parity, &own);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(

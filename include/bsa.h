@@ -119,6 +119,19 @@ int bsa_plan_info(const bsa_plan* plan, int64_t* N, int64_t* nb, int64_t* rows);
 int bsa_plan_set_schedule(bsa_plan* plan, int schedule);
 
 /*
+ * Host-only: the bound, in nanoseconds, of every wait the attention kernels
+ * make inside their main loops (a pipeline stage waiting for a tile, an MMA
+ * or the softmax of another role); 4e9 (4 s) by default.  A wait that runs
+ * out records BSA_EDEVICE in the plan's error word and the kernel stops
+ * early; the output of that call is then unspecified, and the CTAs still
+ * wait for their own tile copies and MMAs before they exit, so the device
+ * stays usable and later calls work normally.  0 makes every wait that is not
+ * already satisfied run out at once (for testing that path).  Takes effect at
+ * the next bsa_attn_run / bsa_attn_run_fp8v / bsa_sparse_attn call.
+ */
+int bsa_plan_set_wait_limit(bsa_plan* plan, uint64_t ns);
+
+/*
  * Host-only: the single-GPU analogue of the review's imbalance factor (Eq.
  * 2, rho = max load / mean load) for one work list: the load of a CTA is
  * the number of key blocks of the items the attention kernel assigns to it
@@ -139,8 +152,8 @@ int bsa_schedule_balance(const bsa_plan* plan, const int32_t* row_ptr, const int
 int bsa_token_order(int T, int Hs, int Ws, int order, int32_t* perm);
 
 /* Bytes of device workspace that bsa_route (BSA_OP_ROUTE), bsa_sparse_attn
- * and bsa_sparse_attn_fp8v (BSA_OP_ATTN), bsa_mask_window_anchor
- * (BSA_OP_MASK) or bsa_augment (BSA_OP_AUGMENT) need; 0 for a NULL plan or
+ * and bsa_sparse_attn_fp8v (BSA_OP_ATTN), bsa_mask_window_anchor and
+ * bsa_mask_stripes_device (BSA_OP_MASK) or bsa_augment (BSA_OP_AUGMENT) need; 0 for a NULL plan or
  * an unknown op. */
 size_t bsa_workspace_size(const bsa_plan* plan, int op);
 
@@ -181,7 +194,10 @@ int bsa_route(const bsa_plan* plan, const void* q, const void* k, int dtype,
  * shape fits, the 720p one does not).  The plan's device must be current.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) and caches it, so make that first call before any
- * stream capture begins.  All calls share the one array: calls that overlap
+ * stream capture begins.  The cached address belongs to the device's primary
+ * context: after cudaDeviceReset (or anything else that destroys that
+ * context) it is stale, so do not call bsa_route_static again in the same
+ * process after such a reset.  All calls share the one array: calls that overlap
  * on the GPU (two streams, or two threads) race and must be serialised by the
  * caller.  Nothing in the array needs to start at zero.  Allocates nothing.
  */
@@ -325,6 +341,21 @@ int bsa_mask_window_anchor(const bsa_plan* plan, int radius_frames, int n_anchor
  */
 int bsa_mask_stripes(int B, int H, int T, int Hs, int Ws, int block, int order, const int32_t* params,
                      int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, int64_t* nnz);
+
+/*
+ * The same stripe masks produced on the device, for a plan (the plan's B, H,
+ * token order, block and grid; PSA pages, section 3.2 "Efficient and Flexible
+ * Kernel": the masks are applied per block inside the attention kernel's
+ * pipeline, so here they are written straight into device memory).  params:
+ * HOST int32 [H][6] as for bsa_mask_stripes, H <= 160 (BSA_EUNSUPPORTED
+ * above), copied into the launch.  Outputs: DEVICE row_ptr int32 [rows+1],
+ * col_idx int32 [col_cap] (columns ascending), nnz int64 (device) = the full
+ * count; BSA_ECAPACITY in the device error word if it exceeds col_cap
+ * (columns past col_cap are dropped).  workspace: >= bsa_workspace_size(plan,
+ * BSA_OP_MASK) bytes, 256-aligned.  Identical CSR to bsa_mask_stripes.
+ */
+int bsa_mask_stripes_device(const bsa_plan* plan, const int32_t* params, int32_t* row_ptr, int32_t* col_idx,
+                            int64_t col_cap, int64_t* nnz, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Block-sparse attention (the pages' "Block-Sparse Attention Execution"):

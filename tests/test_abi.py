@@ -92,6 +92,8 @@ def test_null_plan_calls(bsa):
     assert bsa._lib.bsa_last_device_error(None, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_plan_info(None, None, None, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_plan_set_schedule(None, 0) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_plan_set_wait_limit(None, 0) == bsa.BSA_EINVAL
+    assert bsa._lib.bsa_mask_stripes_device(None, None, None, None, 0, None, None, 0, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_schedule_balance(None, None, None, None, None, None) == bsa.BSA_EINVAL
     assert bsa._lib.bsa_attn_intermediates(None, None, None, None, None) == bsa.BSA_EINVAL
 

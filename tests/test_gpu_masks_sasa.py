@@ -118,3 +118,47 @@ def test_augment_matches_oracle(bsa, cid, extras):
     assert checked > 0.9 * plan.rows
     heads_ok = ~skip.reshape(heads, nb).any(axis=1)
     assert np.allclose(L_o.cpu().numpy()[heads_ok], L_ref[heads_ok], rtol=0, atol=1e-6)
+
+
+def _stripe_params(rng, H):
+    return [(int(rng.integers(0, 3)), int(rng.integers(-3, 4)), int(rng.integers(-1, 6)),
+             int(rng.integers(0, 4)), int(rng.integers(-4, 5)), int(rng.integers(-1, 8))) for _ in range(H)]
+
+
+def gpu_stripes(bsa, w, params, order=0, col_cap=None):
+    plan = bsa.Plan(w.B, w.H, w.T, w.Hs, w.Ws, w.d, w.block, order)
+    cap = plan.rows * plan.nb if col_cap is None else col_cap
+    rp = torch.empty(plan.rows + 1, dtype=torch.int32, device="cuda")
+    ci = torch.full((max(cap, 1),), -1, dtype=torch.int32, device="cuda")
+    nnz = torch.empty(1, dtype=torch.int64, device="cuda")
+    ws = plan.workspace(bsa.BSA_OP_MASK)
+    rc = bsa.bsa_mask_stripes_device(plan, params, rp, ci, cap, nnz, ws)
+    return rc, rp.cpu().numpy(), ci.cpu().numpy(), int(nnz.item()), bsa.bsa_last_device_error(plan)
+
+
+@pytest.mark.parametrize("shape", [(4, 2, 2, 64, 1, 1), (6, 8, 10, 64, 1, 3), (5, 9, 7, 128, 2, 2),
+                                   (21, 30, 52, 128, 1, 12)])
+@pytest.mark.parametrize("order", [0, 1])
+def test_stripes_device_matches_oracle(bsa, shape, order):
+    """PSA stripe masks made on the device equal the oracle's CSR exactly (the last
+    shape is the 480p workload with twelve random heads)."""
+    import oracle.stripes as ostr
+    T, Hs, Ws, block, B, H = shape
+    w = syn.workload(2, T=T, Hs=Hs, Ws=Ws, block=block, B=B, H=H)
+    params = _stripe_params(np.random.default_rng(T * 100 + Hs + order), H)
+    rc, rp, ci, nnz, st = gpu_stripes(bsa, w, params, order)
+    assert rc == 0 and st == 0
+    want_rp, want_ci = ostr.stripe_csr(B, H, T, Hs, Ws, block, np.array(params),
+                                       order="hilbert" if order == 0 else "identity")
+    np.testing.assert_array_equal(rp, want_rp)
+    assert nnz == want_ci.size
+    np.testing.assert_array_equal(ci[:nnz], want_ci)
+
+
+def test_stripes_device_capacity_and_errors(bsa):
+    w = syn.workload(2, T=6, Hs=8, Ws=10, block=64, H=1)
+    rc, rp, ci, nnz, st = gpu_stripes(bsa, w, [(0, 0, 0, 8, 0, 0)], col_cap=3)
+    assert rc == 0 and st == bsa.BSA_ECAPACITY and nnz > 3 and rp[-1] == nnz
+    assert gpu_stripes(bsa, w, [(-1, 0, 0, 0, 0, 0)])[0] == bsa.BSA_EINVAL
+    w2 = syn.workload(2, T=1, Hs=8, Ws=8, block=64, H=161)
+    assert gpu_stripes(bsa, w2, [(0, 0, 0, 0, 0, 0)] * 161)[0] == bsa.BSA_EUNSUPPORTED

@@ -147,3 +147,22 @@ def test_too_many_blocks_unsupported(bsa):
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
     assert bsa.bsa_route(plan, d, d, bsa.BSA_F32, 0.9, 1, d, d, 0, d, torch.empty(1, dtype=torch.int64, device="cuda"),
                          ws) == bsa.BSA_EUNSUPPORTED
+
+
+@pytest.mark.parametrize("case", ["flat", "outlier", "two_clusters"])
+def test_bucket_sort_on_skewed_rows(bsa, case):
+    """Rows of more than 256 blocks go through the bucket sort: every score in one
+    bucket (all scores equal), a single far outlier squeezing the rest into few
+    buckets, and two distant clusters -- masks still match the oracle."""
+    w = syn.workload(1, T=8, Hs=40, Ws=60, H=2)            # fp32 inputs, nb = 300 > 256
+    x = syn.make_inputs(w, seed=19)
+    perm = oracle.token_perm(w.T, w.Hs, w.Ws)
+    if case == "flat":
+        x["q"][:] = 0.0                                    # every block score is 0
+    elif case == "outlier":
+        x["k"][:, perm[:w.block]] *= 200.0                 # key block 0 far above the rest
+        x["q"][:, perm[:w.block]] *= 200.0
+    else:
+        x["k"][:, perm[: w.N // 2]] += 30.0                # half the key blocks shifted far away
+    compare(bsa, w, x, 0.9, 3)
+    compare(bsa, w, x, 0.5, 0)

@@ -123,3 +123,62 @@ def test_balance_step(world, hpr, skew, policy):
         assert got == list(want)
     else:
         assert all(all(e == 0 for e in res[r][3]) for r in range(world))
+
+
+def _exec_worker(rank, world, port, hpr, skew, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import block_sparse_attention_top_b200 as bsa
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        heads = list(range(rank * hpr, (rank + 1) * hpr))
+        g = torch.Generator().manual_seed(11 + rank)
+        L = (torch.rand(hpr, generator=g) * 4 + 10 + (skew if rank == 0 else 0.0)).tolist()
+        # Q, K, V of a head hold its id in every element (K = 2 id, V = 3 id)
+        qx = torch.stack([torch.full((1, 4, 2), float(h)) for h in heads], dim=2)
+        kx, vx = 2 * qx, 3 * qx
+
+        def compute(q2, k2, v2, heads_now, extra):
+            # the stand-in for route + attention on this rank: output of head h = 1000 h + its extra
+            # blocks + a check that its Q, K, V arrived together (h, 2h, 3h)
+            out = torch.empty_like(q2)
+            for i, h in enumerate(heads_now):
+                same = bool(torch.all(q2[:, :, i] == h) and torch.all(k2[:, :, i] == 2 * h)
+                            and torch.all(v2[:, :, i] == 3 * h))
+                out[:, :, i] = 1000.0 * h + extra[i] + (0.0 if same else 0.5)
+            return out
+
+        o, st = bsa.balanced_attention(qx, kx, vx, L, heads, rank, world, compute)
+        q.put((rank, o[0, 0, :, 0].tolist(), st["moves"], st["local_heads"], st["extra"], st["policy"]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,hpr,skew", [(2, 3, 30.0), (4, 2, 40.0), (4, 3, 0.0)])
+def test_balanced_attention_restores_head_order(world, hpr, skew):
+    """Rank-local execution after the migration, then the reverse migration: each rank gets back the
+    outputs of its own heads, in its original head order, computed from that head's Q, K and V and
+    with the augmentation the plan gave the rank that computed it."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_exec_worker, args=(r, world, port, hpr, skew, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {r[0]: r[1:] for r in (q.get(timeout=120) for _ in range(world))}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    moves = res[0][1]
+    if skew > 0:
+        assert moves                                          # something moved
+    extra_of = {}
+    for r in range(world):
+        for h, e in zip(res[r][2], res[r][3]):
+            extra_of[h] = e                                   # extra of the rank that computed h
+    for r in range(world):
+        home = list(range(r * hpr, (r + 1) * hpr))
+        assert res[r][0] == [1000.0 * h + extra_of[h] for h in home]
