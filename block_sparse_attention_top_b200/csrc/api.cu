@@ -141,12 +141,13 @@ int bsa_plan_create(bsa_plan** out, int B, int H, int T, int Hs, int Ws,
     p->wait_ns = 4000000000ull;
     std::vector<int32_t> perm((size_t)N);
     token_order(T, Hs, Ws, order, perm.data());
-    if (cudaMalloc(&p->d_perm, (size_t)N * sizeof(int32_t)) != cudaSuccess ||
-        cudaMalloc(&p->d_err, 4 * sizeof(int32_t)) != cudaSuccess ||
-        cudaMemcpy(p->d_perm, perm.data(), (size_t)N * sizeof(int32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemset(p->d_err, 0, 4 * sizeof(int32_t)) != cudaSuccess) {
-        cudaFree(p->d_perm); cudaFree(p->d_err);
-        delete p;
+    const bool ok = cudaMalloc(&p->d_perm, (size_t)N * sizeof(int32_t)) == cudaSuccess &&
+                    cudaMalloc(&p->d_err, 4 * sizeof(int32_t)) == cudaSuccess &&
+                    cudaMemcpy(p->d_perm, perm.data(), (size_t)N * sizeof(int32_t), cudaMemcpyHostToDevice) ==
+                        cudaSuccess &&
+                    cudaMemset(p->d_err, 0, 4 * sizeof(int32_t)) == cudaSuccess;
+    if (!ok) {
+        bsa_plan_destroy(p);
         return BSA_ECUDA;
     }
     *out = p;
@@ -255,9 +256,7 @@ int bsa_route(const bsa_plan* p, const void* q, const void* k, int dtype, float 
     double* scores = (double*)(base + L.scores);
     uint16_t* sorted = (uint16_t*)(base + L.sorted);
     int32_t* counts = (int32_t*)(base + L.counts);
-    BSA_LAUNCH(launch_pool(*p, q, k, dtype, qbar, kbar, s));
-    BSA_LAUNCH(launch_scores(*p, qbar, kbar, scores, s));
-    BSA_LAUNCH(launch_route_rows(*p, scores, (double)pval, k_floor, sorted, counts, s));
+    BSA_LAUNCH(launch_route_stages(*p, q, k, dtype, (double)pval, k_floor, qbar, kbar, scores, sorted, counts, s));
     BSA_LAUNCH(launch_csr(*p, counts, sorted, row_ptr, col_idx, col_cap, L_h, nnz, s));
     return BSA_OK;
 }

@@ -49,12 +49,19 @@ __device__ __forceinline__ void record_error(int32_t* err, int status, int detai
 }
 
 // ---- launchers (return cudaError_t of the launch) ----
+// The routing stages of bsa_route / bsa_route_static (pool, scores, row
+// routing) into the given scratch on `s`; the CSR stage follows.
+cudaError_t launch_route_stages(const bsa_plan& p, const void* q, const void* k, int dtype, double pval, int k_floor,
+                                double* qbar, double* kbar, double* scores, uint16_t* sorted, int32_t* counts,
+                                cudaStream_t s);
+// Routing stages over heads h0 .. h0 + nh - 1 of every batch entry (nh <= 0:
+// through the last head).
 cudaError_t launch_pool(const bsa_plan& p, const void* q, const void* k, int dtype,
-                        double* qbar, double* kbar, cudaStream_t s);
+                        double* qbar, double* kbar, cudaStream_t s, int h0 = 0, int nh = 0);
 cudaError_t launch_scores(const bsa_plan& p, const double* qbar, const double* kbar,
-                          double* scores, cudaStream_t s);
+                          double* scores, cudaStream_t s, int h0 = 0, int nh = 0);
 cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pval, int k_floor,
-                              uint16_t* sorted, int32_t* counts, cudaStream_t s);
+                              uint16_t* sorted, int32_t* counts, cudaStream_t s, int h0 = 0, int nh = 0);
 cudaError_t launch_csr(const bsa_plan& p, const int32_t* counts, const uint16_t* sorted,
                        int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, float* L_h,
                        int64_t* nnz, cudaStream_t s);

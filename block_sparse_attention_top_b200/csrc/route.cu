@@ -3,10 +3,11 @@
 // a Top-k safety floor; L_h from the review's Eq. 1).
 //
 //   k_pool       gather through the token order + block mean of Q and K (HBM bound)
-//   k_scores     s_ij = <Qbar_i, Kbar_j> / sqrt(d), register-tiled fp64
-//   k_route_warp softmax, sort by (P desc, j asc), cumulative mass, Top-p cut,
-//   k_route_cta  Top-k floor -> count and importance order per row (one warp
-//                per row up to 256 blocks, one CTA per row above)
+//   k_scores_mma s_ij = <Qbar_i, Kbar_j> / sqrt(d), fp64 MMA (m8n8k4)
+//   k_route_warp   softmax, sort by (P desc, j asc), cumulative mass, Top-p
+//   k_route_bucket cut, Top-k floor -> count and importance order per row
+//   k_route_cta    (one warp per row up to 256 blocks, an exact bucket sort
+//                  per row up to 4096, a CTA bitonic sort above)
 //   k_csr_scan   exclusive scan of the counts -> row_ptr, nnz, L_h
 //   k_csr_fill   copy each row's kept columns into col_idx
 //
@@ -20,6 +21,15 @@
 
 namespace bsa {
 namespace {
+
+// The heads a launch covers: h0 .. h0 + nh - 1 of every batch entry.  Local
+// head t (0 <= t < B * nh) is (b, h) = (t / nh, h0 + t % nh); local row l of
+// a launch over rows is (local head l / nb, query block l % nb).
+struct HeadRange {
+    int H, h0, nh;
+    __device__ __forceinline__ int bh(int t) const { return (t / nh) * H + h0 + t % nh; }
+    __device__ __forceinline__ int64_t row(int64_t l, int nb) const { return (int64_t)bh((int)(l / nb)) * nb + l % nb; }
+};
 
 // ---------------------------------------------------------------------------
 // Pooling: one CTA per (query/key tensor, batch, block, 64 chunks of the H*d
@@ -59,7 +69,8 @@ template <> struct Vec16<float> {
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restrict__ perm,
-       double* __restrict__ qbar, double* __restrict__ kbar, int N, int H, int d, int block, int nb) {
+       double* __restrict__ qbar, double* __restrict__ kbar, int N, int H, int d, int block, int nb, int chunk0,
+       int chunk_end) {
     constexpr int V = Vec16<T>::n;
     __shared__ int32_t s_tok[128];
     __shared__ double part[kPoolGroups - 1][kPoolChunks][V];
@@ -75,8 +86,8 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
 
     const int hd = H * d;
     const int g = threadIdx.x / kPoolChunks;
-    const int c = blockIdx.y * kPoolChunks + threadIdx.x % kPoolChunks;   // 16-byte chunk within the row
-    const bool live = c * V < hd;
+    const int c = chunk0 + blockIdx.y * kPoolChunks + threadIdx.x % kPoolChunks;   // 16-byte chunk of the row
+    const bool live = c < chunk_end;
     const uint4* base = reinterpret_cast<const uint4*>(x + (size_t)b * N * hd) + c;
     const size_t row_stride = (size_t)hd / V;              // in uint4
 
@@ -90,6 +101,7 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
 #pragma unroll
             for (int r = 0; r < kPoolUnroll; ++r)
                 u[r] = __ldg(base + (size_t)s_tok[t + kPoolGroups * r] * row_stride);
+            asm volatile("" ::: "memory");          // every load of the batch is issued before any is used
 #pragma unroll
             for (int r = 0; r < kPoolUnroll; ++r) {
                 double w[V];
@@ -125,87 +137,7 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Scores: TM x TM output tile per CTA (TM = 64 or 128), 256 threads, each
-// (TM/16) x (TM/16) outputs held in registers; d consumed in slices of 16
-// staged through shared memory; fp64 FMA.
-// ---------------------------------------------------------------------------
-constexpr int kSK = 16;
-
-template <int TM>
-__global__ void __launch_bounds__(256)
-k_scores(const double* __restrict__ qbar, const double* __restrict__ kbar, double* __restrict__ S,
-         int nb, int d, double scale) {
-    constexpr int R = TM / 16;
-    constexpr int L = TM * kSK / 256;                 // elements of each operand loaded per thread per slice
-    extern __shared__ double score_smem[];             // [2 operands][2 buffers][kSK][TM + 1]
-    auto As = reinterpret_cast<double (*)[kSK][TM + 1]>(score_smem);
-    auto Bs = reinterpret_cast<double (*)[kSK][TM + 1]>(score_smem + 2 * kSK * (TM + 1));
-    const int bh = blockIdx.z;
-    const int i0 = blockIdx.y * TM, j0 = blockIdx.x * TM;
-    const double* Q = qbar + (size_t)bh * nb * d;
-    const double* K = kbar + (size_t)bh * nb * d;
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    double acc[R][R];
-#pragma unroll
-    for (int u = 0; u < R; ++u)
-#pragma unroll
-        for (int v = 0; v < R; ++v) acc[u][v] = 0.0;
-    // slice loads: element e = threadIdx.x + 256*l -> (row e / 16, column e % 16); 16 threads read one
-    // row's 128 contiguous bytes
-    double pa[L], pb[L];
-    auto fetch = [&](int k0) {
-#pragma unroll
-        for (int l = 0; l < L; ++l) {
-            const int e = threadIdx.x + 256 * l, rr = e / kSK, kk = e % kSK;
-            pa[l] = (i0 + rr < nb) ? Q[(size_t)(i0 + rr) * d + k0 + kk] : 0.0;
-            pb[l] = (j0 + rr < nb) ? K[(size_t)(j0 + rr) * d + k0 + kk] : 0.0;
-        }
-    };
-    auto stash = [&](int buf) {
-#pragma unroll
-        for (int l = 0; l < L; ++l) {
-            const int e = threadIdx.x + 256 * l, rr = e / kSK, kk = e % kSK;
-            As[buf][kk][rr] = pa[l];
-            Bs[buf][kk][rr] = pb[l];
-        }
-    };
-    fetch(0);
-    stash(0);
-    __syncthreads();
-    int buf = 0;
-    for (int k0 = 0; k0 < d; k0 += kSK) {
-        const bool more = k0 + kSK < d;
-        if (more) fetch(k0 + kSK);                    // in flight while this slice is multiplied
-#pragma unroll
-        for (int kk = 0; kk < kSK; ++kk) {
-            double av[R], bv[R];
-#pragma unroll
-            for (int u = 0; u < R; ++u) { av[u] = As[buf][kk][ty + 16 * u]; bv[u] = Bs[buf][kk][tx + 16 * u]; }
-#pragma unroll
-            for (int u = 0; u < R; ++u)
-#pragma unroll
-                for (int v = 0; v < R; ++v) acc[u][v] = fma(av[u], bv[v], acc[u][v]);
-        }
-        if (more) stash(buf ^ 1);                     // the other buffer was last read one slice ago
-        __syncthreads();
-        buf ^= 1;
-    }
-    double* out = S + (size_t)bh * nb * nb;
-#pragma unroll
-    for (int u = 0; u < R; ++u) {
-        const int i = i0 + ty + 16 * u;
-        if (i >= nb) continue;
-#pragma unroll
-        for (int v = 0; v < R; ++v) {
-            const int j = j0 + tx + 16 * v;
-            if (j < nb) out[(size_t)i * nb + j] = acc[u][v] * scale;
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Scores on the FP64 MMA path (mma.sync m8n8k4 .f64: fp64 products and sums,
-// the same precision as the FMA kernel above, a different summation order).
+// Scores on the FP64 MMA path (mma.sync m8n8k4 .f64: fp64 products and sums).
 // CTA tile 64 x 64 of one head, 4 warps of 32 x 32 (4 x 4 tiles of 8 x 8);
 // Qbar and Kbar staged in slices of 16 along d, double-buffered.  Fragments
 // of m8n8k4: A (8x4) a0 = A[lane/4][lane%4]; B (4x8) b0 = B[lane%4][lane/4];
@@ -221,12 +153,12 @@ __device__ __forceinline__ void dmma(double& c0, double& c1, double a, double b)
                  : "d"(a), "d"(b));
 }
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 4)
 k_scores_mma(const double* __restrict__ qbar, const double* __restrict__ kbar, double* __restrict__ S, int nb,
-             int d, double scale) {
+             int d, double scale, HeadRange hr) {
     __shared__ double As[2][kMT][kMLd];
     __shared__ double Bs[2][kMT][kMLd];
-    const int bh = blockIdx.z;
+    const int bh = hr.bh(blockIdx.z);
     const int i0 = blockIdx.y * kMT, j0 = blockIdx.x * kMT;
     const double* Q = qbar + (size_t)bh * nb * d;
     const double* K = kbar + (size_t)bh * nb * d;
@@ -325,13 +257,14 @@ __device__ __forceinline__ double key_score(unsigned long long key) {
 template <int E>
 __global__ void __launch_bounds__(128, 1)
 k_route_warp(const double* __restrict__ S, int64_t rows, int nb, double p, int k_floor,
-             uint16_t* __restrict__ sorted, int32_t* __restrict__ counts) {
+             uint16_t* __restrict__ sorted, int32_t* __restrict__ counts, HeadRange hr) {
     constexpr int NBP = 32 * E;
     constexpr int LOGN = E == 1 ? 5 : E == 2 ? 6 : E == 4 ? 7 : E == 8 ? 8 : E == 16 ? 9 : 10;
     static_assert((1 << LOGN) == NBP, "E must be a power of two <= 32");
     const int lane = threadIdx.x % 32;
-    const int64_t r = (int64_t)blockIdx.x * 4 + threadIdx.x / 32;
-    if (r >= rows) return;
+    const int64_t lr = (int64_t)blockIdx.x * 4 + threadIdx.x / 32;
+    if (lr >= rows) return;
+    const int64_t r = hr.row(lr, nb);
     const double* row = S + r * nb;
     unsigned long long key[E];
     double mx = -INFINITY;
@@ -431,7 +364,7 @@ constexpr int kCtaSortThreads = 256;
 template <int E>
 __global__ void __launch_bounds__(kCtaSortThreads)
 k_route_cta(const double* __restrict__ S, int nb, double p, int k_floor,
-            uint16_t* __restrict__ sorted, int32_t* __restrict__ counts) {
+            uint16_t* __restrict__ sorted, int32_t* __restrict__ counts, HeadRange hr) {
     constexpr int NBP = kCtaSortThreads * E;
     constexpr int LOGN = E == 2 ? 9 : E == 4 ? 10 : E == 8 ? 11 : E == 16 ? 12 : 13;
     static_assert((1 << LOGN) == NBP, "E must be 2, 4, 8, 16 or 32");
@@ -439,7 +372,7 @@ k_route_cta(const double* __restrict__ S, int nb, double p, int k_floor,
     __shared__ double red[kCtaSortThreads / 32];
     __shared__ int s_first;
     const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
-    const size_t r = blockIdx.x;
+    const size_t r = (size_t)hr.row(blockIdx.x, nb);
     const double* row = S + r * nb;
     unsigned long long key[E];
     double mx = -INFINITY;
@@ -594,19 +527,23 @@ __device__ __forceinline__ double block_max(double v, double* red) {
     return t;
 }
 
-// dynamic shared memory: keys [nb] u64, placed [nb] u64, count [NB] int, start [NB] int
+// dynamic shared memory: keys [nb] u64, placed [nb] u64, pj [nb] f64 (exp(s_j - max)),
+// bucket [nb] int, count [NB] int, start [NB] int
 __global__ void __launch_bounds__(kBucketThreads)
 k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_floor,
-               uint16_t* __restrict__ sorted, int32_t* __restrict__ counts) {
+               uint16_t* __restrict__ sorted, int32_t* __restrict__ counts, HeadRange hr) {
     extern __shared__ unsigned long long bsm[];
     unsigned long long* keys = bsm;
     unsigned long long* placed = bsm + nb;
-    int* cnt = reinterpret_cast<int*>(bsm + 2 * nb);
+    double* pj = reinterpret_cast<double*>(bsm + 2 * nb);
+    int* bucket = reinterpret_cast<int*>(bsm + 3 * nb);
+    int* cnt = bucket + nb;
     int* start = cnt + NB;
     __shared__ double red[kBucketThreads / 32];
+    __shared__ int wsum[kBucketThreads / 32];
     __shared__ int s_first;
-    const int tid = threadIdx.x;
-    const size_t r = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
+    const size_t r = (size_t)hr.row(blockIdx.x, nb);
     const double* row = S + r * nb;
 
     double mx = -INFINITY, mn = INFINITY;
@@ -615,6 +552,7 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
         mx = fmax(mx, sv);
         mn = fmin(mn, sv);
         keys[j] = desc_key(sv, j);
+        pj[j] = sv;
     }
     for (int b = tid; b < NB; b += kBucketThreads) cnt[b] = 0;
     if (tid == 0) s_first = nb;
@@ -622,16 +560,17 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
     mn = -block_max(-mn, red);
     const double width = mx - mn;
     const double to_bucket = width > 0.0 ? (double)NB / width : 0.0;
-    // bucket counts; each key keeps its arrival slot only to be placed somewhere in its bucket
+    // bucket of each score (monotone in s), the unnormalised mass exp(s - max) of its key
     double zpart = 0.0;
     for (int j = tid; j < nb; j += kBucketThreads) {
-        const double sv = key_score(keys[j]);
-        zpart += exp(sv - mx);
-        const int b = min(NB - 1, (int)((mx - row[j]) * to_bucket));
+        const int b = min(NB - 1, (int)((mx - pj[j]) * to_bucket));
+        bucket[j] = b;
+        const double e = exp(key_score(keys[j]) - mx);
+        pj[j] = e;
+        zpart += e;
         atomicAdd(&cnt[b], 1);
     }
     const double z = block_sum(zpart, red);
-    __syncthreads();
     // exclusive scan of the counts (NB / 128 per thread, then across the block)
     {
         const int per = NB / kBucketThreads;
@@ -639,13 +578,11 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
         int run = 0;
         for (int u = 0; u < per; ++u) run += cnt[lo + u];
         int incl = run;
-        const int lane = tid % 32, wid = tid / 32;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        __shared__ int wsum[kBucketThreads / 32];
         if (lane == 31) wsum[wid] = incl;
         __syncthreads();
         int off = incl - run;
@@ -658,14 +595,14 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
     }
     __syncthreads();
     for (int j = tid; j < nb; j += kBucketThreads) {
-        const int b = min(NB - 1, (int)((mx - row[j]) * to_bucket));
+        const int b = bucket[j];
         placed[start[b] + atomicAdd(&cnt[b], 1)] = keys[j];
     }
     __syncthreads();
     // each key's final place: its bucket's start + the number of smaller keys in the bucket
     for (int q = tid; q < nb; q += kBucketThreads) {
         const unsigned long long key = placed[q];
-        const int b = min(NB - 1, (int)((mx - row[(int)(key & kJMask)]) * to_bucket));
+        const int b = bucket[(int)(key & kJMask)];
         const int b0 = start[b], b1 = b0 + cnt[b];
         int rank = b0;
         for (int u = b0; u < b1; ++u) rank += placed[u] < key;
@@ -673,12 +610,12 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
     }
     __syncthreads();
     // P in sorted order, inclusive cumulative mass (contiguous chunks per thread), first n with C_n >= p
+    const double inv_z = 1.0 / z;
     const int per = (nb + kBucketThreads - 1) / kBucketThreads;
     const int q0 = tid * per, q1 = min(nb, q0 + per);
     double run = 0.0;
-    for (int q = q0; q < q1; ++q) run += exp(key_score(keys[q]) - mx) / z;
+    for (int q = q0; q < q1; ++q) run += pj[(int)(keys[q] & kJMask)] * inv_z;
     double incl = run;
-    const int lane = tid % 32, wid = tid / 32;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const double y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -690,7 +627,7 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
     for (int w = 0; w < wid; ++w) c += red[w];
     int first = nb;
     for (int q = q0; q < q1; ++q) {
-        c += exp(key_score(keys[q]) - mx) / z;
+        c += pj[(int)(keys[q] & kJMask)] * inv_z;
         if (c >= p) { first = q + 1; break; }
     }
 #pragma unroll
@@ -773,73 +710,91 @@ __global__ void k_csr_fill(const int32_t* __restrict__ counts, const uint16_t* _
 }  // namespace
 
 cudaError_t launch_pool(const bsa_plan& p, const void* q, const void* k, int dtype,
-                        double* qbar, double* kbar, cudaStream_t s) {
+                        double* qbar, double* kbar, cudaStream_t s, int h0, int nh) {
+    if (nh <= 0) nh = p.H - h0;
     const int V = dtype == BSA_BF16 ? 8 : 4;
-    const int chunks = (p.H * p.d) / V;
-    dim3 grid((unsigned)p.nb, (unsigned)((chunks + kPoolChunks - 1) / kPoolChunks), (unsigned)(2 * p.B));
+    const int c0 = h0 * p.d / V, c1 = (h0 + nh) * p.d / V;     // chunks of heads h0 .. h0 + nh - 1
+    dim3 grid((unsigned)p.nb, (unsigned)((c1 - c0 + kPoolChunks - 1) / kPoolChunks), (unsigned)(2 * p.B));
     if (dtype == BSA_BF16)
         k_pool<__nv_bfloat16><<<grid, kPoolThreads, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                                             p.d_perm, qbar, kbar, (int)p.N, p.H, p.d, p.block,
-                                                            (int)p.nb);
+                                                            (int)p.nb, c0, c1);
     else
         k_pool<float><<<grid, kPoolThreads, 0, s>>>((const float*)q, (const float*)k, p.d_perm, qbar, kbar,
-                                                    (int)p.N, p.H, p.d, p.block, (int)p.nb);
-    return cudaGetLastError();
-}
-
-template <int TM>
-cudaError_t launch_scores_tm(const bsa_plan& p, const double* qbar, const double* kbar, double* scores,
-                             cudaStream_t s, double scale) {
-    const int smem = 4 * kSK * (TM + 1) * (int)sizeof(double);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_scores<TM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-    }
-    const int t = (int)((p.nb + TM - 1) / TM);
-    dim3 grid(t, t, (unsigned)(p.B * p.H));
-    k_scores<TM><<<grid, 256, smem, s>>>(qbar, kbar, scores, (int)p.nb, p.d, scale);
+                                                    (int)p.N, p.H, p.d, p.block, (int)p.nb, c0, c1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_scores(const bsa_plan& p, const double* qbar, const double* kbar, double* scores,
-                          cudaStream_t s) {
+                          cudaStream_t s, int h0, int nh) {
+    if (nh <= 0) nh = p.H - h0;
     const double scale = 1.0 / sqrt((double)p.d);
-    if (p.d % kMK == 0) {
-        const int t = (int)((p.nb + kMT - 1) / kMT);
-        dim3 grid(t, t, (unsigned)(p.B * p.H));
-        k_scores_mma<<<grid, 128, 0, s>>>(qbar, kbar, scores, (int)p.nb, p.d, scale);
-        return cudaGetLastError();
-    }
-    const int64_t t128 = (p.nb + 127) / 128;
-    if (t128 * t128 * p.B * p.H >= 2 * p.num_sms) return launch_scores_tm<128>(p, qbar, kbar, scores, s, scale);
-    return launch_scores_tm<64>(p, qbar, kbar, scores, s, scale);
+    const int t = (int)((p.nb + kMT - 1) / kMT);            // d (64 or 128) is a multiple of the d slice
+    dim3 grid(t, t, (unsigned)(p.B * nh));
+    k_scores_mma<<<grid, 128, 0, s>>>(qbar, kbar, scores, (int)p.nb, p.d, scale, HeadRange{p.H, h0, nh});
+    return cudaGetLastError();
 }
 
 cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pval, int k_floor,
-                              uint16_t* sorted, int32_t* counts, cudaStream_t s) {
+                              uint16_t* sorted, int32_t* counts, cudaStream_t s, int h0, int nh) {
+    if (nh <= 0) nh = p.H - h0;
+    const HeadRange hr{p.H, h0, nh};
+    const int64_t rows = (int64_t)p.B * nh * p.nb;
     int nbp = 1;
     while (nbp < p.nb) nbp <<= 1;
     nbp = nbp < 2 ? 2 : nbp;
     const int nb = (int)p.nb;
     if (nbp <= 256) {
-        const unsigned grid = (unsigned)((p.rows + 3) / 4);
+        const unsigned grid = (unsigned)((rows + 3) / 4);
         switch (nbp <= 32 ? 1 : nbp / 32) {
-            case 1: k_route_warp<1><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
-            case 2: k_route_warp<2><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
-            case 4: k_route_warp<4><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
-            default: k_route_warp<8><<<grid, 128, 0, s>>>(scores, p.rows, nb, pval, k_floor, sorted, counts); break;
+            case 1: k_route_warp<1><<<grid, 128, 0, s>>>(scores, rows, nb, pval, k_floor, sorted, counts, hr); break;
+            case 2: k_route_warp<2><<<grid, 128, 0, s>>>(scores, rows, nb, pval, k_floor, sorted, counts, hr); break;
+            case 4: k_route_warp<4><<<grid, 128, 0, s>>>(scores, rows, nb, pval, k_floor, sorted, counts, hr); break;
+            default: k_route_warp<8><<<grid, 128, 0, s>>>(scores, rows, nb, pval, k_floor, sorted, counts, hr); break;
         }
         return cudaGetLastError();
     }
-    // exact bucket sort: NB = 2 * nbp buckets, at most 8192 (a multiple of the block size)
-    const int NB = 2 * nbp < 8192 ? 2 * nbp : 8192;
-    const size_t smem = (size_t)2 * nb * sizeof(unsigned long long) + (size_t)2 * NB * sizeof(int);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_route_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
+    if (nbp <= 4096) {
+        // exact bucket sort: NB = nbp buckets (a multiple of the block size)
+        const int NB = nbp;
+        const size_t smem = (size_t)3 * nb * sizeof(unsigned long long) + (size_t)(nb + 2 * NB) * sizeof(int);
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(k_route_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        k_route_bucket<<<(unsigned)rows, kBucketThreads, smem, s>>>(scores, nb, NB, pval, k_floor, sorted, counts, hr);
+        return cudaGetLastError();
     }
-    k_route_bucket<<<(unsigned)p.rows, kBucketThreads, smem, s>>>(scores, nb, NB, pval, k_floor, sorted, counts);
-    return cudaGetLastError();
+    // longer rows: CTA bitonic sort (E keys per thread)
+    const int E = nbp / kCtaSortThreads;
+    const size_t smem = (size_t)nbp * sizeof(unsigned long long);
+    auto run = [&](auto kern) -> cudaError_t {
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        kern<<<(unsigned)rows, kCtaSortThreads, smem, s>>>(scores, nb, pval, k_floor, sorted, counts, hr);
+        return cudaGetLastError();
+    };
+    switch (E) {
+        case 2: return run(k_route_cta<2>);
+        case 4: return run(k_route_cta<4>);
+        case 8: return run(k_route_cta<8>);
+        case 16: return run(k_route_cta<16>);
+        default: return run(k_route_cta<32>);
+    }
+}
+
+cudaError_t launch_route_stages(const bsa_plan& p, const void* q, const void* k, int dtype, double pval, int k_floor,
+                                double* qbar, double* kbar, double* scores, uint16_t* sorted, int32_t* counts,
+                                cudaStream_t s) {
+    // one pass over all heads per stage (splitting heads into groups and running
+    // pooling of one group beside the scores and sorts of another on a second
+    // stream measured slower at 480p and 720p)
+    cudaError_t e = launch_pool(p, q, k, dtype, qbar, kbar, s);
+    if (e == cudaSuccess) e = launch_scores(p, qbar, kbar, scores, s);
+    if (e == cudaSuccess) e = launch_route_rows(p, scores, pval, k_floor, sorted, counts, s);
+    return e;
 }
 
 cudaError_t launch_scan_counts(const bsa_plan& p, const int32_t* counts, int32_t* row_ptr, float* L_h,

@@ -73,9 +73,9 @@ extern "C" int bsa_route_static(const bsa_plan* p, const void* q, const void* k,
     double* scores = (double*)(base + L.scores);
     uint16_t* sorted = (uint16_t*)(base + L.sorted);
     int32_t* counts = (int32_t*)(base + L.counts);
-    if (launch_pool(*p, q, k, dtype, qbar, kbar, s) != cudaSuccess) return BSA_ECUDA;
-    if (launch_scores(*p, qbar, kbar, scores, s) != cudaSuccess) return BSA_ECUDA;
-    if (launch_route_rows(*p, scores, (double)pval, k_floor, sorted, counts, s) != cudaSuccess) return BSA_ECUDA;
+    if (launch_route_stages(*p, q, k, dtype, (double)pval, k_floor, qbar, kbar, scores, sorted, counts, s) !=
+        cudaSuccess)
+        return BSA_ECUDA;
     if (launch_csr(*p, counts, sorted, row_ptr, col_idx, col_cap, L_h, nnz, s) != cudaSuccess) return BSA_ECUDA;
     return BSA_OK;
 }

@@ -69,6 +69,8 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
     }
 }
 // Bounded wait: false if the abort flag is raised or the time limit passes.
+// (Every waiter spins: a pause between probes, even only in the producer and
+// MMA warps, measured 15 % slower.)
 template <uint32_t kEvery = 1023>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl) {
     return mbar_test(bar, parity) || mbar_wait_slow<kEvery>(bar, parity, ctl);
