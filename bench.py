@@ -140,7 +140,10 @@ ATTN_SOURCES = ("attn_pp.cu", "tc_common.cuh")
 # DRAM bytes (read + write) of one k_attn_pp launch on the headline workload, from one
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the sha256 of
 # the kernel sources it was taken on; a kernel built from other sources reports null.
-ATTN_TRAFFIC = {}
+ATTN_TRAFFIC = {
+    # 12-head 720p capture (2.391 GB per launch) scaled by retained work to the 40-head launch
+    "79c4f2f28dde88246a5942c15b7f66ed82c90ea8c20ebac703f7c81803654067": 7956400089,
+}
 SCHEDULES = (("l2_heads", 0), ("heaviest_first", 1), ("in_order", 2))
 
 
