@@ -5,9 +5,10 @@
 //   k_pool       gather through the token order + block mean of Q and K (HBM bound)
 //   k_scores_mma s_ij = <Qbar_i, Kbar_j> / sqrt(d), fp64 MMA (m8n8k4)
 //   k_route_warp   softmax, sort by (P desc, j asc), cumulative mass, Top-p
-//   k_route_bucket cut, Top-k floor -> count and importance order per row
-//   k_route_cta    (one warp per row up to 256 blocks, an exact bucket sort
-//                  per row up to 4096, a CTA bitonic sort above)
+//   k_route_bwarp  cut, Top-k floor -> count and importance order per row
+//   k_route_bucket (a register bitonic sort per warp up to 256 blocks, an
+//   k_route_cta    exact bucket sort per warp up to 1024 and per CTA up to
+//                  4096, a CTA bitonic sort above)
 //   k_csr_scan   exclusive scan of the counts -> row_ptr, nnz, L_h
 //   k_csr_fill   copy each row's kept columns into col_idx
 //
@@ -28,7 +29,11 @@ namespace {
 struct HeadRange {
     int H, h0, nh;
     __device__ __forceinline__ int bh(int t) const { return (t / nh) * H + h0 + t % nh; }
-    __device__ __forceinline__ int64_t row(int64_t l, int nb) const { return (int64_t)bh((int)(l / nb)) * nb + l % nb; }
+    // rows of a launch fit int32 (the library rejects rows * nb >= 2^31), so 32-bit division
+    __device__ __forceinline__ int64_t row(int64_t l, int nb) const {
+        const int l32 = (int)l, t = l32 / nb;
+        return (int64_t)bh(t) * nb + (l32 - t * nb);
+    }
 };
 
 // ---------------------------------------------------------------------------
@@ -145,7 +150,8 @@ k_pool(const T* __restrict__ q, const T* __restrict__ k, const int32_t* __restri
 // ---------------------------------------------------------------------------
 constexpr int kMT = 64;                  // CTA tile (rows and columns)
 constexpr int kMK = 16;                  // d slice
-constexpr int kMLd = kMK + 1;            // padded shared row (doubles)
+constexpr int kMLd = kMK + 4;            // shared row of 20 doubles: a half-warp's fragment reads
+                                         // (rows g, columns t) and 16-byte stores hit distinct banks
 
 __device__ __forceinline__ void dmma(double& c0, double& c1, double a, double b) {
     asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
@@ -156,8 +162,8 @@ __device__ __forceinline__ void dmma(double& c0, double& c1, double a, double b)
 __global__ void __launch_bounds__(128, 4)
 k_scores_mma(const double* __restrict__ qbar, const double* __restrict__ kbar, double* __restrict__ S, int nb,
              int d, double scale, HeadRange hr) {
-    __shared__ double As[2][kMT][kMLd];
-    __shared__ double Bs[2][kMT][kMLd];
+    __shared__ __align__(16) double As[2][kMT][kMLd];
+    __shared__ __align__(16) double Bs[2][kMT][kMLd];
     const int bh = hr.bh(blockIdx.z);
     const int i0 = blockIdx.y * kMT, j0 = blockIdx.x * kMT;
     const double* Q = qbar + (size_t)bh * nb * d;
@@ -185,12 +191,13 @@ k_scores_mma(const double* __restrict__ qbar, const double* __restrict__ kbar, d
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
             const int e = tid + 128 * l, r = e / (kMK / 2), c2 = e % (kMK / 2);
-            As[buf][r][2 * c2] = ra[l].x;
-            As[buf][r][2 * c2 + 1] = ra[l].y;
-            Bs[buf][r][2 * c2] = rb[l].x;
-            Bs[buf][r][2 * c2 + 1] = rb[l].y;
+            *reinterpret_cast<double2*>(&As[buf][r][2 * c2]) = ra[l];
+            *reinterpret_cast<double2*>(&Bs[buf][r][2 * c2]) = rb[l];
         }
     };
+    // a warp whose 32 x 32 quarter lies wholly outside [0, nb) (in the ragged last tile row
+    // or column) only helps to stage the slices
+    const bool live = i0 + wm < nb && j0 + wn < nb;
     fetch(0);
     stash(0);
     __syncthreads();
@@ -198,18 +205,20 @@ k_scores_mma(const double* __restrict__ qbar, const double* __restrict__ kbar, d
     for (int k0 = 0; k0 < d; k0 += kMK) {
         const bool more = k0 + kMK < d;
         if (more) fetch(k0 + kMK);                    // in flight while this slice is multiplied
+        if (live) {
 #pragma unroll
-        for (int ks = 0; ks < kMK / 4; ++ks) {
-            double av[4], bv[4];
+            for (int ks = 0; ks < kMK / 4; ++ks) {
+                double av[4], bv[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                av[u] = As[buf][wm + 8 * u + g][4 * ks + t];
-                bv[u] = Bs[buf][wn + 8 * u + g][4 * ks + t];
+                for (int u = 0; u < 4; ++u) {
+                    av[u] = As[buf][wm + 8 * u + g][4 * ks + t];
+                    bv[u] = Bs[buf][wn + 8 * u + g][4 * ks + t];
+                }
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) dmma(acc[mt][nt][0], acc[mt][nt][1], av[mt], bv[nt]);
             }
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) dmma(acc[mt][nt][0], acc[mt][nt][1], av[mt], bv[nt]);
         }
         if (more) stash(buf ^ 1);                     // the other buffer was last read one slice ago
         __syncthreads();
@@ -642,6 +651,161 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
 }
 
 // ---------------------------------------------------------------------------
+// Row routing by a warp-level exact bucket sort (rows of 257 to 1024 blocks):
+// one warp per row, four rows per CTA, no CTA barrier.  Lane l keeps the keys
+// of blocks l, l + 32, l + 64, ... in registers (the 64-bit keys above).  Each
+// key goes to bucket floor((max - s) * NB / (max - min)), monotone in s,
+// through a histogram of 16-bit counts in shared memory whose atomic add also
+// returns the key's slot inside its bucket.  A warp scan turns the counts into
+// bucket starts, the keys are scattered to their buckets, each key's rank is
+// its bucket's start plus the number of smaller keys in the bucket, and the
+// keys are rewritten in place in rank order.  The exponentials exp(s - max),
+// their running sum in sorted order (a contiguous run of C keys per lane, C
+// odd so that the lanes' 64-bit reads fall on distinct banks), the total z
+// and the first n with sum_{k<=n} e_k >= p z follow in fp64.
+// ---------------------------------------------------------------------------
+constexpr int kBwarpRows = 4;
+
+__device__ __forceinline__ int bucket_start(const uint32_t* bw, int b) {
+    return (int)((bw[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu);
+}
+
+// per-warp shared memory: keys [nb] u64, then NB / 2 + 1 words of two 16-bit
+// counts (later starts; start[NB] = nb)
+__host__ __device__ __forceinline__ int bwarp_stride(int nb, int NB) { return nb + (NB / 2 + 2) / 2; }
+
+template <int E>
+__global__ void __launch_bounds__(32 * kBwarpRows)
+k_route_bwarp(const double* __restrict__ S, int64_t rows, int nb, int NB, double p, int k_floor,
+              uint16_t* __restrict__ sorted, int32_t* __restrict__ counts, HeadRange hr) {
+    extern __shared__ unsigned long long wsm[];
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    const int64_t lr = (int64_t)blockIdx.x * kBwarpRows + wid;
+    if (lr >= rows) return;                               // the whole warp; nothing waits on it
+    unsigned long long* keys = wsm + (size_t)wid * bwarp_stride(nb, NB);
+    uint32_t* bw = reinterpret_cast<uint32_t*>(keys + nb);
+    const int64_t r = hr.row(lr, nb);
+    const double* row = S + r * nb;
+
+    unsigned long long key[E];
+    double mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = lane + 32 * e;
+        key[e] = 0;
+        if (j < nb) {
+            key[e] = desc_key(row[j], j);
+            const double sv = key_score(key[e]);
+            mx = fmax(mx, sv);
+            mn = fmin(mn, sv);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    for (int w = lane; w <= NB / 2; w += 32) bw[w] = 0;
+    __syncwarp();
+    // bucket of each key and its slot inside the bucket (arrival order, refined below)
+    const double width = mx - mn;
+    const double to_bucket = width > 0.0 ? (double)NB / width : 0.0;
+    uint32_t slot[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        slot[e] = 0;
+        if (lane + 32 * e < nb) {
+            const int b = min(NB - 1, (int)((mx - key_score(key[e])) * to_bucket));
+            const int sh = (b & 1) * 16;
+            const uint32_t old = atomicAdd(&bw[b >> 1], 1u << sh);
+            slot[e] = (uint32_t)b | (((old >> sh) & 0xFFFFu) << 16);
+        }
+    }
+    __syncwarp();
+    // exclusive scan of the counts: lane l owns words [l W, l W + W), W = NB / 64
+    {
+        const int W = NB / 64;
+        uint32_t run = 0;
+        for (int w = 0; w < W; ++w) {
+            const uint32_t v = bw[lane * W + w];
+            run += (v & 0xFFFFu) + (v >> 16);
+        }
+        uint32_t incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        uint32_t off = incl - run;
+        for (int w = 0; w < W; ++w) {
+            const uint32_t v = bw[lane * W + w];
+            const uint32_t s0 = off, s1 = off + (v & 0xFFFFu);
+            off = s1 + (v >> 16);
+            bw[lane * W + w] = s0 | (s1 << 16);
+        }
+        if (lane == 31) bw[NB / 2] = (uint32_t)nb;        // start[NB] = nb
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (lane + 32 * e < nb) keys[bucket_start(bw, (int)(slot[e] & 0xFFFFu)) + (int)(slot[e] >> 16)] = key[e];
+    __syncwarp();
+    // each key's rank: its bucket's start + the smaller keys in the bucket
+    int rk[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        rk[e] = 0;
+        if (lane + 32 * e < nb) {
+            const int b = (int)(slot[e] & 0xFFFFu);
+            const int b0 = bucket_start(bw, b), b1 = bucket_start(bw, b + 1);
+            int rank = b0;
+            for (int u = b0; u < b1; ++u) rank += keys[u] < key[e];
+            rk[e] = rank;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (lane + 32 * e < nb) keys[rk[e]] = key[e];
+    __syncwarp();
+    uint16_t* dst = sorted + r * nb;
+    for (int q = lane; q < nb; q += 32) dst[q] = (uint16_t)(keys[q] & kJMask);   // the full importance order
+    __syncwarp();
+    // exponentials in sorted order (each lane a contiguous run of C keys, written over
+    // its own keys), their running sum, then the Top-p cut
+    const int C = ((nb + 31) / 32) | 1;
+    const int q0 = min(nb, lane * C), q1 = min(nb, q0 + C);
+    double* ex = reinterpret_cast<double*>(keys);
+    double run = 0.0;
+    for (int q = q0; q < q1; ++q) {
+        const double e = exp(key_score(keys[q]) - mx);
+        ex[q] = e;
+        run += e;
+    }
+    double incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const double target = p * __shfl_sync(0xffffffffu, incl, 31);
+    double c = incl - run;
+    int first = nb;
+    for (int q = q0; q < q1; ++q) {
+        c += ex[q];
+        if (c >= target) {
+            first = q + 1;
+            break;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    const int n_p = p >= 1.0 ? nb : first;
+    const int n_i = min(nb, max(k_floor, n_p));
+    if (lane == 0) counts[r] = n_i;
+}
+
+// ---------------------------------------------------------------------------
 // CSR: single-CTA exclusive scan of the counts, then a row-parallel copy.
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 1024;
@@ -753,6 +917,24 @@ cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pv
             default: k_route_warp<8><<<grid, 128, 0, s>>>(scores, rows, nb, pval, k_floor, sorted, counts, hr); break;
         }
         return cudaGetLastError();
+    }
+    if (nbp <= 1024) {
+        // warp-level exact bucket sort: NB = nbp / 2 buckets, E >= ceil(nb / 32) keys per lane (odd)
+        const int NB = nbp / 2;
+        const size_t smem = (size_t)kBwarpRows * bwarp_stride(nb, NB) * sizeof(unsigned long long);
+        const unsigned grid = (unsigned)((rows + kBwarpRows - 1) / kBwarpRows);
+        const int need = ((nb + 31) / 32) | 1;
+        auto run = [&](auto kern) -> cudaError_t {
+            if (smem > 48 * 1024) {
+                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (e != cudaSuccess) return e;
+            }
+            kern<<<grid, 32 * kBwarpRows, smem, s>>>(scores, rows, nb, NB, pval, k_floor, sorted, counts, hr);
+            return cudaGetLastError();
+        };
+        if (need <= 13) return run(k_route_bwarp<13>);
+        if (need <= 21) return run(k_route_bwarp<21>);
+        return run(k_route_bwarp<33>);
     }
     if (nbp <= 4096) {
         // exact bucket sort: NB = nbp buckets (a multiple of the block size)

@@ -83,8 +83,10 @@ def test_ragged_shapes(bsa, shape, order):
 
 
 @pytest.mark.parametrize("shape", [
-    dict(T=8, Hs=100, Ws=100, H=1, d=64, block=64),     # 1250 blocks per row: CTA sort, 8 keys per thread
-    dict(T=26, Hs=100, Ws=101, H=1, d=64, block=64),    # 4104 blocks per row: CTA sort, 32 keys per thread
+    dict(T=4, Hs=80, Ws=80, H=2, d=64, block=64),       # 400 blocks per row: warp bucket sort, 13 keys per lane
+    dict(T=4, Hs=125, Ws=127, H=2, d=64, block=64),     # 993 blocks per row (ragged): warp bucket sort, 33 keys per lane
+    dict(T=8, Hs=100, Ws=100, H=1, d=64, block=64),     # 1250 blocks per row: CTA bucket sort
+    dict(T=26, Hs=100, Ws=101, H=1, d=64, block=64),    # 4104 blocks per row: CTA bitonic sort, 32 keys per thread
 ])
 def test_long_rows(bsa, shape):
     w = syn.workload(2, **shape)
