@@ -641,13 +641,16 @@ k_route_bucket(const double* __restrict__ S, int nb, int NB, double p, int k_flo
 // ---------------------------------------------------------------------------
 constexpr int kBwarpRows = 4;
 
-__device__ __forceinline__ int bucket_start(const uint32_t* bw, int b) {
-    return (int)((bw[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu);
+// Word of bucket pair w (buckets 2w, 2w + 1): one pad word after every NB / 64
+// words, so that the lanes' contiguous ranges in the scan start on distinct banks.
+__device__ __forceinline__ int bucket_word(int w, int NB) { return w + (w >> (__ffs(NB) - 7)); }
+__device__ __forceinline__ int bucket_start(const uint32_t* bw, int b, int NB) {
+    return (int)((bw[bucket_word(b >> 1, NB)] >> ((b & 1) * 16)) & 0xFFFFu);
 }
 
-// per-warp shared memory: keys [nb] u64, then NB / 2 + 1 words of two 16-bit
-// counts (later starts; start[NB] = nb)
-__host__ __device__ __forceinline__ int bwarp_stride(int nb, int NB) { return nb + (NB / 2 + 2) / 2; }
+// per-warp shared memory: keys [nb] u64, then NB / 2 + 33 words of two 16-bit
+// counts (later starts; start[NB] = nb) with the pad words
+__host__ __device__ __forceinline__ int bwarp_stride(int nb, int NB) { return nb + (NB / 2 + 34) / 2; }
 
 template <int E>
 __global__ void __launch_bounds__(32 * kBwarpRows)
@@ -680,7 +683,7 @@ k_route_bwarp(const double* __restrict__ S, int64_t rows, int nb, int NB, double
         mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
-    for (int w = lane; w <= NB / 2; w += 32) bw[w] = 0;
+    for (int w = lane; w <= NB / 2 + 32; w += 32) bw[w] = 0;
     __syncwarp();
     // bucket of each key and its slot inside the bucket (arrival order, refined below)
     const double width = mx - mn;
@@ -692,17 +695,17 @@ k_route_bwarp(const double* __restrict__ S, int64_t rows, int nb, int NB, double
         if (lane + 32 * e < nb) {
             const int b = min(NB - 1, (int)((mx - key_score(key[e])) * to_bucket));
             const int sh = (b & 1) * 16;
-            const uint32_t old = atomicAdd(&bw[b >> 1], 1u << sh);
+            const uint32_t old = atomicAdd(&bw[bucket_word(b >> 1, NB)], 1u << sh);
             slot[e] = (uint32_t)b | (((old >> sh) & 0xFFFFu) << 16);
         }
     }
     __syncwarp();
-    // exclusive scan of the counts: lane l owns words [l W, l W + W), W = NB / 64
+    // exclusive scan of the counts: lane l owns words [l (W + 1), l (W + 1) + W), W = NB / 64
     {
         const int W = NB / 64;
         uint32_t run = 0;
         for (int w = 0; w < W; ++w) {
-            const uint32_t v = bw[lane * W + w];
+            const uint32_t v = bw[lane * (W + 1) + w];
             run += (v & 0xFFFFu) + (v >> 16);
         }
         uint32_t incl = run;
@@ -713,17 +716,17 @@ k_route_bwarp(const double* __restrict__ S, int64_t rows, int nb, int NB, double
         }
         uint32_t off = incl - run;
         for (int w = 0; w < W; ++w) {
-            const uint32_t v = bw[lane * W + w];
+            const uint32_t v = bw[lane * (W + 1) + w];
             const uint32_t s0 = off, s1 = off + (v & 0xFFFFu);
             off = s1 + (v >> 16);
-            bw[lane * W + w] = s0 | (s1 << 16);
+            bw[lane * (W + 1) + w] = s0 | (s1 << 16);
         }
-        if (lane == 31) bw[NB / 2] = (uint32_t)nb;        // start[NB] = nb
+        if (lane == 31) bw[bucket_word(NB / 2, NB)] = (uint32_t)nb;     // start[NB] = nb
     }
     __syncwarp();
 #pragma unroll
     for (int e = 0; e < E; ++e)
-        if (lane + 32 * e < nb) keys[bucket_start(bw, (int)(slot[e] & 0xFFFFu)) + (int)(slot[e] >> 16)] = key[e];
+        if (lane + 32 * e < nb) keys[bucket_start(bw, (int)(slot[e] & 0xFFFFu), NB) + (int)(slot[e] >> 16)] = key[e];
     __syncwarp();
     // each key's rank: its bucket's start + the smaller keys in the bucket
     int rk[E];
@@ -732,7 +735,7 @@ k_route_bwarp(const double* __restrict__ S, int64_t rows, int nb, int NB, double
         rk[e] = 0;
         if (lane + 32 * e < nb) {
             const int b = (int)(slot[e] & 0xFFFFu);
-            const int b0 = bucket_start(bw, b), b1 = bucket_start(bw, b + 1);
+            const int b0 = bucket_start(bw, b, NB), b1 = bucket_start(bw, b + 1, NB);
             int rank = b0;
             for (int u = b0; u < b1; ++u) rank += keys[u] < key[e];
             rk[e] = rank;
@@ -895,8 +898,9 @@ cudaError_t launch_route_rows(const bsa_plan& p, const double* scores, double pv
         return cudaGetLastError();
     }
     if (nbp <= 1024) {
-        // warp-level exact bucket sort: NB = nbp / 2 buckets, E >= ceil(nb / 32) keys per lane (odd)
-        const int NB = nbp / 2;
+        // warp-level exact bucket sort: NB = 2 nbp buckets (2048 at 591 blocks: 12 us faster
+        // than 512 there), E >= ceil(nb / 32) keys per lane (odd)
+        const int NB = 2 * nbp;
         const size_t smem = (size_t)kBwarpRows * bwarp_stride(nb, NB) * sizeof(unsigned long long);
         const unsigned grid = (unsigned)((rows + kBwarpRows - 1) / kBwarpRows);
         const int need = ((nb + 31) / 32) | 1;
