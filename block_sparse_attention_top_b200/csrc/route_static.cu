@@ -1,7 +1,6 @@
 // bsa_route_static: the routing entry point for callers that cannot allocate
 // device memory when they route -- for example a host that has handed all
-// device memory to its own fixed arena or caching allocator, or code that
-// runs while a stream capture is active, where cudaMalloc is not allowed.
+// device memory to its own fixed arena or caching allocator.
 //
 // It runs exactly the kernels of bsa_route, but their scratch (pooled Q/K,
 // block scores, sorted indices, counts) lives in one file-scope device array

@@ -183,9 +183,8 @@ int bsa_route(const bsa_plan* plan, const void* q, const void* k, int dtype,
 
 /*
  * bsa_route without a workspace argument, for callers that cannot allocate
- * device memory at the time they route: a host whose device memory is all
- * owned by its own arena or caching allocator, or code running while a stream
- * capture is active, where cudaMalloc is not allowed.  The FVAttn pages have
+ * device memory at the time they route, such as a host whose device memory is
+ * all owned by its own arena or caching allocator.  The FVAttn pages have
  * no counterpart to this call; it only changes where the scratch lives.
  * Same arguments, results and errors as bsa_route.  The scratch is one
  * library-owned device array of 32 MiB, held by every GPU that loads the
@@ -193,13 +192,13 @@ int bsa_route(const bsa_plan* plan, const void* q, const void* k, int dtype,
  * BSA_OP_ROUTE) exceeds it are rejected with BSA_EWORKSPACE (e.g. the 480p
  * shape fits, the 720p one does not).  The plan's device must be current.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it, so make that first call before any
- * stream capture begins.  The cached address belongs to the device's primary
- * context: after cudaDeviceReset (or anything else that destroys that
- * context) it is stale, so do not call bsa_route_static again in the same
- * process after such a reset.  All calls share the one array: calls that overlap
- * on the GPU (two streams, or two threads) race and must be serialised by the
- * caller.  Nothing in the array needs to start at zero.  Allocates nothing.
+ * (cudaGetSymbolAddress) and caches it.  The cached address belongs to the
+ * device's primary context: after cudaDeviceReset (or anything else that
+ * destroys that context) it is stale, so do not call bsa_route_static again
+ * in the same process after such a reset.  All calls share the one array:
+ * calls that overlap on the GPU (two streams, or two threads) race and must
+ * be serialised by the caller.  Nothing in the array needs to start at zero.
+ * Allocates nothing.
  */
 int bsa_route_static(const bsa_plan* plan, const void* q, const void* k, int dtype,
                      float p, int k_floor,

@@ -1,8 +1,7 @@
 """The allocation-free routing entry point (bsa_route_static).
 
 Some callers cannot allocate device memory when they route -- their device
-memory belongs to their own arena, or they are inside a stream capture where
-cudaMalloc is not allowed.  bsa_route_static serves them from a fixed device
+memory belongs to their own arena.  bsa_route_static serves them from a fixed device
 array owned by the library.  These tests call it through the C ABI twice in a
 row, on different inputs, and require the same masks, L_h and nnz as
 bsa_route with a caller workspace (bit-exact, the routing tolerance).  The
