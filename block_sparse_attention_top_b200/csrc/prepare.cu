@@ -24,6 +24,8 @@
 // [block, d] tile the attention kernel can fetch with a single TMA box.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -115,25 +117,38 @@ __global__ void k_iota(const int32_t* __restrict__ row_ptr, int64_t rows, int nb
     work[r] = (int32_t)r;
 }
 
-// One thread moves 16 bytes.  Destination rows are visited in (b, n', h)
-// order so that consecutive threads read one token's contiguous H*d row.
-__global__ void k_permute(const uint4* __restrict__ q, const uint4* __restrict__ k,
-                          const uint4* __restrict__ v, uint4* __restrict__ qp, uint4* __restrict__ kp,
-                          uint4* __restrict__ vp, const int32_t* __restrict__ perm, int N, int H,
-                          int vec_per_row, int64_t npad, int64_t total) {
-    const uint4* src = blockIdx.y == 0 ? q : (blockIdx.y == 1 ? k : v);
-    uint4* dst = blockIdx.y == 0 ? qp : (blockIdx.y == 1 ? kp : vp);
-    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
-         g += (int64_t)gridDim.x * blockDim.x) {
-        const int c = (int)(g % vec_per_row);
-        int64_t rest = g / vec_per_row;
-        const int h = (int)(rest % H);
-        rest /= H;
-        const int64_t n = rest % npad;
-        const int64_t b = rest / npad;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (n < N) val = __ldg(src + ((b * N + perm[n]) * H + h) * vec_per_row + c);
-        dst[((b * H + h) * npad + n) * vec_per_row + c] = val;
+// One CTA per kPermRows consecutive destination rows n of the padded sequence
+// (and batch entry, tensor): each row copies token perm[n]'s contiguous H*d row
+// into the H per-head tiles (zeros for the padding rows n >= N).  Thread t moves
+// the 16-byte chunks t, t + blockDim, ... of the row, the loads of the CTA's
+// rows in flight together; a head's rows land as one contiguous run.
+constexpr int kPermRows = 4;
+
+__global__ void __launch_bounds__(1024)
+k_permute(const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+          uint4* __restrict__ qp, uint4* __restrict__ kp, uint4* __restrict__ vp, const int32_t* __restrict__ perm,
+          int N, int H, int vec_per_row, int64_t npad) {
+    const int b = blockIdx.y;
+    const uint4* src = blockIdx.z == 0 ? q : (blockIdx.z == 1 ? k : v);
+    uint4* dst = blockIdx.z == 0 ? qp : (blockIdx.z == 1 ? kp : vp);
+    const int row_vecs = H * vec_per_row;
+    int64_t n[kPermRows], srow[kPermRows];
+    bool real[kPermRows];
+#pragma unroll
+    for (int r = 0; r < kPermRows; ++r) {
+        n[r] = (int64_t)blockIdx.x * kPermRows + r;
+        real[r] = n[r] < N;
+        srow[r] = real[r] ? ((int64_t)b * N + perm[n[r]]) * row_vecs : 0;
+    }
+    for (int e = threadIdx.x; e < row_vecs; e += blockDim.x) {
+        const int h = e / vec_per_row, c = e - h * vec_per_row;
+        uint4 val[kPermRows];
+#pragma unroll
+        for (int r = 0; r < kPermRows; ++r) val[r] = real[r] ? __ldg(src + srow[r] + e) : make_uint4(0u, 0u, 0u, 0u);
+        uint4* out = dst + ((int64_t)b * H + h) * npad * vec_per_row + c;
+#pragma unroll
+        for (int r = 0; r < kPermRows; ++r)
+            if (n[r] < npad) out[n[r] * vec_per_row] = val[r];
     }
 }
 
@@ -187,14 +202,11 @@ cudaError_t launch_permute(const bsa_plan& p, const void* q, const void* k, cons
                            void* kp, void* vp, cudaStream_t s, int n_tensors) {
     const int vec_per_row = p.d * 2 / 16;
     const int64_t npad = p.nb * p.block;
-    const int64_t total = (int64_t)p.B * npad * p.H * vec_per_row;
-    const int t = 256;
-    int64_t blocks = (total + t - 1) / t;
-    const int64_t cap = (int64_t)p.num_sms * 16;
-    if (blocks > cap) blocks = cap;
-    dim3 grid((unsigned)blocks, (unsigned)n_tensors);
+    const int row_vecs = p.H * vec_per_row;
+    const int t = std::min(1024, (row_vecs + 31) / 32 * 32);
+    const dim3 grid((unsigned)((npad + kPermRows - 1) / kPermRows), (unsigned)p.B, (unsigned)n_tensors);
     k_permute<<<grid, t, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (uint4*)qp, (uint4*)kp,
-                                 (uint4*)vp, p.d_perm, (int)p.N, p.H, vec_per_row, npad, total);
+                                 (uint4*)vp, p.d_perm, (int)p.N, p.H, vec_per_row, npad);
     return cudaGetLastError();
 }
 
