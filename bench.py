@@ -267,6 +267,14 @@ def extra_case(bsa, torch, dev, stream, flush, cid, p_index, n, pk):
     return out
 
 
+def bench_config(w, p_index, world):
+    """The `config` both arms print for the same workload (the reference arm
+    states how it ran in `reference_execution`)."""
+    return {"workload": workload_desc(w, p_index), "global_batch": w.B * world, "seq_len": w.N,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every timed call (256 MB write, untimed)"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import block_sparse_attention_top_b200 as bsa
@@ -435,10 +443,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) + sinusoidal (t,y,x) features, Wan-shaped video latents; no weights)",
-        "config": {"workload": workload_desc(w, args.p_index), "global_batch": w.B * world, "seq_len": w.N,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed before every timed call (256 MB write, untimed)",
-                   "density": round(density, 4)},
+        "config": bench_config(w, args.p_index, world),
+        "density": round(density, 4),
         "attn_ms_per_call": round(attn_avg, 4),
         "attn_tflops": round(achieved, 2),
         "attn_frac_of_bf16_burst": round(achieved / pk["bf16_tflops"], 4),
@@ -557,9 +563,9 @@ def run_reference(args, world=1):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(w, args.p_index), "global_batch": w.B * world, "seq_len": w.N,
-                       "parallelism": "CPU oracle (numpy fp64)", "l2": "not applicable (host)",
-                       "density": round(density, 4)},
+            "config": bench_config(w, args.p_index, world), "density": round(density, 4),
+            "reference_execution": "the fp64 numpy oracle on the host cores, rank 0 only (no GPU: the config's L2 "
+                                   "flush does not apply)",
             "ms_per_step_kind": "timed: one bounded sample step (oracle routing of one head + attention on one "
                                 "query block); value extrapolates it to the full step's work",
             "full_step_ms_extrapolated": round(full_ms, 2),
